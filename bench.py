@@ -1,0 +1,422 @@
+"""Benchmark of the AB-Attention hot path on B200 (one JSON line on rank 0).
+
+One step = one pass of the whole hot path on the Wan2.1-14B-shaped layer
+(B=1, H=40, N=75,600 = 21x45x80, d=128, KV block 4, s=2048 of 18,900 blocks kept):
+  ab_select(Q, K) -> S, ab_plan(S) -> (idx, logpi), then 4 ab_attn calls on
+  perturbed Q/K/V (sigma 0.05) reusing the plan, as the page reuses a plan for 4
+  denoising steps.
+Inputs are synthetic (random-Fourier Q/K + noise, Gaussian V), generated on the
+device before timing; every tensor is larger than L2, so no flush is needed.
+
+Multi-GPU (torchrun): weak scaling, every rank runs its own full layer (independent
+heads/batches need no exchange); the step time is the max over ranks.
+
+--impl reference times the CPU oracle (the only reference implementation: the pages
+publish no code) on a bounded sample of the same workload, on rank 0.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and kept-block TFLOP/s (% bf16 peak) for ab_attn; select+plan GB/s (% HBM)"
+UNIT = "TFLOP/s"  # kept-block attention FLOPs per second over the whole step
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    import torch
+
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def kept_flops(w):
+    """Kept-block attention FLOPs of one ab_attn call: 4 * B * H * N * (s * bk) * d."""
+    return 4.0 * w.B * w.H * w.N * (w.s * w.kv_block) * w.d
+
+
+def select_plan_bytes(w):
+    """Algorithmic HBM bytes of select+plan: |Q| + |K| (bf16) + 2|S| (fp32) + |idx| + |logpi|."""
+    qk = 2 * w.B * w.H * w.N * w.d * 2
+    S = w.B * w.H * w.nQ * w.nK * 4
+    plan = w.B * w.H * w.nQ * w.s * 8
+    return qk + 2 * S + plan
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import block_sparse_attention_ibcs_b200 as ab
+    from block_sparse_attention_ibcs_b200.inputs import WORKLOADS, make_qkv, perturb
+
+    w = WORKLOADS[args.workload]
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    # each rank runs an independent layer (different seed): weak scaling
+    import dataclasses
+
+    w_r = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    Q, K, V = make_qkv(w_r, device=dev)
+    reuse = max(1, w.plan_reuse)
+    pert = []
+    for c in range(reuse):
+        if w.perturb_sigma > 0:
+            pert.append(tuple(perturb(x, w.perturb_sigma, 7000 + 10 * c + k + 100000 * rank)
+                              for k, x in enumerate((Q, K, V))))
+        else:
+            pert.append((Q, K, V))
+    p = ab.params(w.B, w.H, w.N, w.d, w.kv_block, w.clusters, w.kmeans_iters)
+    rows = w.B * w.H * w.nQ
+    S = torch.empty(w.B, w.H, w.nQ, w.nK, device=dev)
+    ws = torch.empty(ab.ab_workspace_bytes(p), dtype=torch.uint8, device=dev)
+    idx = torch.empty(rows, w.s, dtype=torch.int32, device=dev)
+    lp = torch.empty(rows, w.s, device=dev)
+    Os = [torch.empty_like(Q) for _ in range(reuse)]
+    stream = torch.cuda.current_stream()
+
+    ev = {}
+
+    def E():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(i, record):
+        if record:
+            e0, e1, e2 = E(), E(), E()
+            e0.record(stream)
+        ab.ab_select(p, Q, K, S, ws)
+        if record:
+            e1.record(stream)
+        ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
+        if record:
+            e2.record(stream)
+        att = []
+        for c in range(reuse):
+            qa, ka, va = pert[c]
+            if record:
+                a0, a1 = E(), E()
+                a0.record(stream)
+            ab.ab_attn(p, qa, ka, va, idx, lp, w.s, Os[c])
+            if record:
+                a1.record(stream)
+                att.append((a0, a1))
+        if record:
+            ev.setdefault("steps", []).append((e0, e1, e2, att))
+
+    for i in range(args.warmup):
+        step(i, False)
+    st = ab.ab_get_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {ab.ab_status_string(st)}")
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0, t1 = E(), E()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    st = ab.ab_get_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {ab.ab_status_string(st)}")
+    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    sel_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, e2, _ in ev["steps"])
+    plan_ms = statistics.mean(e1.elapsed_time(e2) for e0, e1, e2, _ in ev["steps"])
+    attn_ms = statistics.mean(a0.elapsed_time(a1) for *_, att in ev["steps"] for a0, a1 in att)
+    F = kept_flops(w)
+    value = world * reuse * F / (ms_step * 1e-3) / 1e12
+    attn_tflops = F / (attn_ms * 1e-3) / 1e12
+    sp_bytes = select_plan_bytes(w)
+    sp_gbs = sp_bytes / ((sel_ms + plan_ms) * 1e-3) / 1e9
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, p, Q, K, pert, reuse, world, dev)
+
+    peak_t = peaks["bf16_tflops_sustained"]
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (random-Fourier Q/K + noise, Gaussian V; seeded)",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({'x'.join(map(str, w.latent))}) "
+                               f"d={w.d} kv_block={w.kv_block} q_block=128 clusters={w.clusters} "
+                               f"s={w.s}/{w.nK} plan_reuse={reuse}",
+                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (Q/K/V 774 MB each), no flush"},
+        "ms_per_attn_call": round(attn_ms, 3),
+        "attn_tflops": round(attn_tflops, 2),
+        "attn_frac_of_bf16_peak": round(attn_tflops / peak_t, 4),
+        "select_ms": round(sel_ms, 3), "plan_ms": round(plan_ms, 3),
+        "select_plan_gbs": round(sp_gbs, 1),
+        "select_plan_frac_of_hbm": round(sp_gbs / peaks["hbm_gbs"], 4),
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,false>",
+                     "achieved": round(attn_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / peak_t, 4),
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained",
+                     "traffic": args.traffic},
+        "gpu_launches": args.steps * (4 + 1 + reuse),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, seconds=args.cpu_seconds)
+    return out
+
+
+def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
+    """Same step through the public API with host inputs: H2D of every input, D2H of every O."""
+    import torch
+
+    import block_sparse_attention_ibcs_b200 as ab
+
+    hostQ, hostK = Q.cpu().pin_memory(), K.cpu().pin_memory()
+    hostP = [tuple(x.cpu().pin_memory() for x in t) for t in pert]
+    hostO = [torch.empty(Q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(reuse)]
+    dQ, dK = torch.empty_like(Q), torch.empty_like(K)
+    dP = [tuple(torch.empty_like(Q) for _ in range(3)) for _ in range(reuse)]
+    rows = w.B * w.H * w.nQ
+    S = torch.empty(w.B, w.H, w.nQ, w.nK, device=dev)
+    ws = torch.empty(ab.ab_workspace_bytes(p), dtype=torch.uint8, device=dev)
+    idx = torch.empty(rows, w.s, dtype=torch.int32, device=dev)
+    lp = torch.empty(rows, w.s, device=dev)
+    dO = [torch.empty_like(Q) for _ in range(reuse)]
+    h2d = (hostQ.numel() + hostK.numel() + 3 * reuse * hostQ.numel()) * 2
+    d2h = reuse * hostQ.numel() * 2
+
+    def step(i):
+        dQ.copy_(hostQ, non_blocking=True)
+        dK.copy_(hostK, non_blocking=True)
+        ab.ab_select(p, dQ, dK, S, ws)
+        ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
+        for c in range(reuse):
+            for dst, src in zip(dP[c], hostP[c]):
+                dst.copy_(src, non_blocking=True)
+            ab.ab_attn(p, dP[c][0], dP[c][1], dP[c][2], idx, lp, w.s, dO[c])
+            hostO[c].copy_(dO[c], non_blocking=True)
+
+    stream = torch.cuda.current_stream()
+    for i in range(2):
+        step(i)
+    steps = max(1, min(args.steps, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(100 + i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    value = world * reuse * kept_flops(w) / (ms * 1e-3) / 1e12
+    return {"value": round(value, 3), "unit": UNIT, "ms_per_step": round(ms, 2), "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def cpu_baseline(w, seconds=15.0):
+    """The oracle as it stands on the host cores: select + plan + attention for a bounded
+    sample of query blocks of head 0, expressed in the metric's unit (kept-block FLOP/s)."""
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_ibcs_b200.inputs import make_qkv
+    from oracle import abattn_oracle as O
+
+    Q, K, V = make_qkv(w, device="cpu", heads=[0])
+    q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
+    cores = torch.get_num_threads()
+    t0 = time.perf_counter()
+    Kp = O.pool_keys(k, w.kv_block)
+    done = 0
+    rows_done = 0
+    qbs = list(range(0, w.nQ, max(1, w.nQ // 64)))
+    for i in qbs:
+        Qb = q[i * 128: min(w.N, (i + 1) * 128)]
+        cent, wt, _, _ = O.kmeans_block(Qb, w.clusters, w.kmeans_iters)
+        S = O.block_scores(cent, wt, Kp).astype(np.float32)
+        idx, lp, _ = O.plan_row(S, w.s, w.philox_seed, 0, i)
+        O.attn_block(Qb, k, v, idx, lp, w.kv_block)
+        done += 1
+        rows_done += Qb.shape[0]
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    flops = 4.0 * rows_done * (w.s * w.kv_block) * w.d
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"head 0, {done} query blocks (select+plan+attn per block, pooling of the "
+                      f"whole head included), {dt:.1f} s",
+            "ms_per_query_block": round(1e3 * dt / done, 1)}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle (the pages publish no implementation)."""
+    if rank != 0:
+        return None
+    from block_sparse_attention_ibcs_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    per = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, seconds=per)
+        if i >= args.warmup:
+            vals.append(cb)
+    value = statistics.mean(c["value"] for c in vals)
+    ms_step = 1e3 * 4.0 * w.B * w.H * w.N * (w.s * w.kv_block) * w.d * max(1, w.plan_reuse) / (value * 1e12)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": f"{w.name} (bounded sample per step, extrapolated)",
+                       "global_batch": w.B, "seq_len": w.N, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan14b")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    out = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,306 @@
+// C ABI of the AB-Attention hot path: argument validation, workspace carving and
+// kernel launches.  All kernels live in the included headers (one translation unit,
+// one device status word).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "abattn.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "plan.cuh"
+#include "select.cuh"
+
+using namespace abattn;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded device wait
+
+bool aligned16(const void* p) { return p != nullptr && ((uintptr_t)p & 15u) == 0; }
+
+int ilog2_exact(int v) {
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return (1 << s) == v ? s : -1;
+}
+
+struct Dims {
+  int B, H, N, d, bk, C, iters;
+  long long BH, nQ, nK;
+};
+
+ab_status check_params(const ab_params* p, Dims* out) {
+  if (!p) return AB_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1 || p->d < 1) return AB_ERR_INVALID_ARG;
+  if (p->kv_block < 1 || p->kv_block > 128 || ilog2_exact(p->kv_block) < 0) return AB_ERR_INVALID_ARG;
+  if (p->clusters < 1 || p->kmeans_iters < 0) return AB_ERR_INVALID_ARG;
+  if (p->q_block != 128) return AB_ERR_UNSUPPORTED;
+  if (p->d != 64 && p->d != 128) return AB_ERR_UNSUPPORTED;
+  if (p->clusters > CMAX || p->kmeans_iters > 4) return AB_ERR_UNSUPPORTED;
+  Dims d;
+  d.B = p->B; d.H = p->H; d.N = p->N; d.d = p->d; d.bk = p->kv_block;
+  d.C = p->clusters; d.iters = p->kmeans_iters;
+  d.BH = (long long)p->B * p->H;
+  d.nQ = (p->N + 127) / 128;
+  d.nK = (p->N + p->kv_block - 1) / p->kv_block;
+  // grid and index limits: every (b,h,query block) is one CTA of a 1-D grid and
+  // element offsets must fit the kernels' size_t arithmetic; nK*2^32 must fit uint64
+  if (d.BH * d.nQ > 0x7fffffffLL || d.nK > (1LL << 30)) return AB_ERR_UNSUPPORTED;
+  *out = d;
+  return AB_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Workspace {
+  uint16_t* Kp;
+  uint16_t* cent;
+  float* w;
+  float* stats;
+  size_t bytes;
+};
+
+Workspace carve(const Dims& d, void* base) {
+  Workspace ws;
+  uint8_t* b = (uint8_t*)base;
+  size_t off = 0;
+  ws.Kp = (uint16_t*)(b + off);
+  off = align256(off + (size_t)d.BH * d.nK * d.d * 2);
+  ws.cent = (uint16_t*)(b + off);
+  off = align256(off + (size_t)d.BH * d.nQ * CMAX * d.d * 2);
+  ws.w = (float*)(b + off);
+  off = align256(off + (size_t)d.BH * d.nQ * CMAX * 4);
+  ws.stats = (float*)(b + off);
+  off = align256(off + (size_t)d.BH * d.nQ * CMAX * 2 * 4);
+  ws.bytes = off;
+  return ws;
+}
+
+ab_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "abattn: CUDA error: %s\n", cudaGetErrorString(e));
+    return AB_ERR_CUDA;
+  }
+  return AB_OK;
+}
+
+template <int D>
+ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, const Workspace& ws,
+                     int8_t* labels, cudaStream_t st) {
+  SelectArgs a;
+  a.Q = (const uint16_t*)Q;
+  a.K = (const uint16_t*)K;
+  a.Kp = ws.Kp;
+  a.cent = ws.cent;
+  a.w = ws.w;
+  a.stats = ws.stats;
+  a.S = S;
+  a.labels = labels;
+  a.BH = (int)d.BH;
+  a.N = d.N;
+  a.nQ = (int)d.nQ;
+  a.nK = (int)d.nK;
+  a.bk = d.bk;
+  a.C = d.C;
+  a.iters = d.iters;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  const size_t units = (size_t)d.BH * d.nK * (D / 8);
+  const int pool_blocks = (int)((units + 255) / 256 < 148 * 32 ? (units + 255) / 256 : 148 * 32);
+  pool_kernel<D><<<pool_blocks, 256, 0, st>>>(a);
+  kmeans_kernel<D><<<(unsigned)(d.BH * d.nQ), KM_THREADS, 0, st>>>(a);
+  const unsigned sc_grid = (unsigned)(d.BH * ((d.nQ + 15) / 16));
+  score_kernel<D, 1><<<sc_grid, SC_THREADS, 0, st>>>(a);
+  score_kernel<D, 2><<<sc_grid, SC_THREADS, 0, st>>>(a);
+  return launch_status();
+}
+
+ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t offset,
+                   int32_t* idx, float* logpi, cudaStream_t st) {
+  PlanArgs a;
+  a.S = S;
+  a.idx = idx;
+  a.logpi = logpi;
+  a.nK = (int)d.nK;
+  a.s = s;
+  a.seed = seed;
+  a.offset = offset;
+  const unsigned rows = (unsigned)(d.BH * d.nQ);
+  if (d.nK <= PLAN_SMEM_MAX_FLOATS) {
+    const size_t smem = (size_t)d.nK * 4;
+    // per-device attribute; cheap enough to set on every launch
+    if (cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PLAN_SMEM_MAX_FLOATS * 4) != cudaSuccess)
+      return launch_status();
+    plan_kernel<true><<<rows, PLAN_THREADS, smem, st>>>(a);
+  } else {
+    plan_kernel<false><<<rows, PLAN_THREADS, 0, st>>>(a);
+  }
+  return launch_status();
+}
+
+template <int D, bool DENSE>
+ab_status run_attn(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
+                   const float* logpi, int s, void* O, int debug_skip, uint64_t timeout_ns,
+                   cudaStream_t st) {
+  AttnArgs a;
+  a.Q = (const uint16_t*)Q;
+  a.K = (const uint16_t*)K;
+  a.V = (const uint16_t*)V;
+  a.idx = idx;
+  a.logpi = logpi;
+  a.O = (uint16_t*)O;
+  a.N = d.N;
+  a.nQ = (int)d.nQ;
+  a.nK = (int)d.nK;
+  a.s = s;
+  a.bk = d.bk;
+  a.bk_shift = ilog2_exact(d.bk);
+  a.ntiles = DENSE ? (int)((d.N + 127) / 128) : (int)(((long long)s * d.bk + 127) / 128);
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  a.timeout_ns = timeout_ns;
+  a.debug_skip_arrive = debug_skip;
+  using L = AttnSmem<D>;
+  if (cudaFuncSetAttribute(attn_kernel<D, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::ALLOC) != cudaSuccess)
+    return launch_status();
+  attn_kernel<D, DENSE><<<(unsigned)(d.BH * d.nQ), ATTN_THREADS, L::ALLOC, st>>>(a);
+  return launch_status();
+}
+
+ab_status attn_common(const ab_params* p, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, const float* logpi, int s, void* O, bool dense,
+                      int debug_skip, uint64_t timeout_ns, void* stream) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return AB_ERR_INVALID_ARG;
+  if (!dense) {
+    if (!idx || !logpi || ((uintptr_t)idx & 3) || ((uintptr_t)logpi & 3)) return AB_ERR_INVALID_ARG;
+    if (s < 1 || s > d.nK) return AB_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (d.d == 128)
+    return dense ? run_attn<128, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st)
+                 : run_attn<128, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st);
+  return dense ? run_attn<64, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st)
+               : run_attn<64, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st);
+}
+
+ab_status select_common(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
+                        size_t ws_bytes, int8_t* labels, void* cent, float* w, void* Kp,
+                        void* stream) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(S)) return AB_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255)) return AB_ERR_WORKSPACE;
+  Workspace wsp = carve(d, ws);
+  if (ws_bytes < wsp.bytes) return AB_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  r = (d.d == 128) ? run_select<128>(d, Q, K, S, wsp, labels, st)
+                   : run_select<64>(d, Q, K, S, wsp, labels, st);
+  if (r != AB_OK) return r;
+  // optional debug copies out of the workspace
+  if (cent) {
+    // [BH, nQ, CMAX, d] -> [BH, nQ, C, d]
+    const size_t row = (size_t)d.d * 2;
+    if (cudaMemcpy2DAsync(cent, row * d.C, wsp.cent, row * CMAX, row * d.C, (size_t)(d.BH * d.nQ),
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return launch_status();
+  }
+  if (w) {
+    if (cudaMemcpy2DAsync(w, 4 * (size_t)d.C, wsp.w, 4 * (size_t)CMAX, 4 * (size_t)d.C,
+                          (size_t)(d.BH * d.nQ), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return launch_status();
+  }
+  if (Kp) {
+    if (cudaMemcpyAsync(Kp, wsp.Kp, (size_t)d.BH * d.nK * d.d * 2, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return launch_status();
+  }
+  return AB_OK;
+}
+
+ab_status plan_common(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
+                      int32_t* idx, float* logpi, void* stream) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!S || !idx || !logpi || ((uintptr_t)S & 3) || ((uintptr_t)idx & 3) || ((uintptr_t)logpi & 3))
+    return AB_ERR_INVALID_ARG;
+  if (s < 1 || s > d.nK) return AB_ERR_INVALID_ARG;
+  return run_plan(d, S, s, seed, offset, idx, logpi, (cudaStream_t)stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+ab_status ab_workspace_bytes(const ab_params* p, size_t* bytes) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!bytes) return AB_ERR_INVALID_ARG;
+  *bytes = carve(d, nullptr).bytes;
+  return AB_OK;
+}
+
+ab_status ab_select(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
+                    size_t ws_bytes, void* stream) {
+  return select_common(p, Q, K, S, ws, ws_bytes, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+ab_status ab_select_debug(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
+                          size_t ws_bytes, int8_t* labels, void* cent, float* w, void* Kp,
+                          void* stream) {
+  return select_common(p, Q, K, S, ws, ws_bytes, labels, cent, w, Kp, stream);
+}
+
+ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
+                  int32_t* idx, float* logpi, void* stream) {
+  return plan_common(p, S, s, seed, offset, idx, logpi, stream);
+}
+
+ab_status ab_sample(const ab_params* p, const float* pi, int s, uint64_t seed, uint64_t offset,
+                    int32_t* idx, float* logpi, void* stream) {
+  return plan_common(p, pi, s, seed, offset, idx, logpi, stream);
+}
+
+ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* V,
+                  const int32_t* idx, const float* logpi, int s, void* O, void* stream) {
+  return attn_common(p, Q, K, V, idx, logpi, s, O, false, 0, kDefaultTimeoutNs, stream);
+}
+
+ab_status ab_attn_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
+                        void* stream) {
+  return attn_common(p, Q, K, V, nullptr, nullptr, 0, O, true, 0, kDefaultTimeoutNs, stream);
+}
+
+ab_status ab_get_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return launch_status();
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_ab_status, sizeof(int)) != cudaSuccess) return launch_status();
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_ab_status, &zero, sizeof(int)) != cudaSuccess) return launch_status();
+  return (ab_status)v;
+}
+
+const char* ab_status_string(ab_status s) {
+  switch (s) {
+    case AB_OK: return "ok";
+    case AB_ERR_INVALID_ARG: return "invalid argument";
+    case AB_ERR_UNSUPPORTED: return "unsupported configuration";
+    case AB_ERR_CUDA: return "CUDA error";
+    case AB_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case AB_ERR_WORKSPACE: return "workspace missing or too small";
+    case AB_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case AB_ERR_DEVICE_CHECK: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+int ab_version(void) { return 100; }
+
+}  // extern "C"

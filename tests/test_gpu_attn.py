@@ -1,0 +1,127 @@
+"""GPU parity of the packed-tile attention (ab_attn, ab_attn_dense) against the fp64 oracle.
+
+Tolerance on O (bf16 inputs, fp32 accumulation, bf16 output, identical plan):
+max-abs <= 1e-2 and relative L2 <= 5e-3.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_ibcs_b200 as ab
+from block_sparse_attention_ibcs_b200.inputs import WORKLOADS, gaussian_head, make_qkv, random_plan
+from oracle import abattn_oracle as O
+
+from _util import assert_o_close, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _qkv(H, N, d, seed):
+    Q = torch.stack([gaussian_head(N, d, seed * 100 + 3 * h) for h in range(H)])[None].bfloat16()
+    K = torch.stack([gaussian_head(N, d, seed * 100 + 3 * h + 1) for h in range(H)])[None].bfloat16()
+    V = torch.stack([gaussian_head(N, d, seed * 100 + 3 * h + 2) for h in range(H)])[None].bfloat16()
+    return Q, K, V
+
+
+def _run(p, Q, K, V, idx, lp, s):
+    O_ = torch.full(Q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    ab.ab_attn(p, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), lp.cuda(), s, O_)
+    assert ab.ab_get_status() == 0
+    return O_
+
+
+def _check(O_gpu, Q, K, V, idx, lp, H, N, bk, qblocks=None):
+    nQ = -(-N // 128)
+    idx = idx.reshape(H, nQ, -1).numpy()
+    lp = lp.reshape(H, nQ, -1).numpy()
+    for h in range(H):
+        Qh, Kh, Vh = np64(Q[0, h]), np64(K[0, h]), np64(V[0, h])
+        Oh = np64(O_gpu[0, h])
+        for i in (range(nQ) if qblocks is None else qblocks):
+            rows = slice(i * 128, min(N, (i + 1) * 128))
+            ref = O.attn_block(Qh[rows], Kh, Vh, idx[h, i], lp[h, i], bk)
+            assert_o_close(Oh[rows], ref, f"h{h} qb{i}")
+
+
+@pytest.mark.parametrize("N,d,bk,s", [
+    (1024, 64, 4, 32),     # tiny config budget: one full tile
+    (1024, 64, 4, 256),    # all blocks (8 tiles)
+    (1000, 64, 4, 33),     # ragged query block (104 rows) + partial tile (132 tokens)
+    (1000, 128, 16, 20),   # d = 128, partial last KV block handled by masking
+    (1000, 64, 64, 9),     # last KV block has 40 valid tokens
+    (1000, 128, 128, 5),   # one block per tile, last block 104 tokens
+    (777, 64, 1, 300),     # single-token blocks, odd N
+    (130, 128, 2, 65),     # two query blocks, the second with 2 rows
+])
+def test_attn_random_plan(N, d, bk, s):
+    H = 2
+    nQ, nK = -(-N // 128), -(-N // bk)
+    Q, K, V = _qkv(H, N, d, seed=N + d + bk)
+    idx, lp = random_plan(H * nQ, nK, s, seed=5)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    O_ = _run(p, Q, K, V, idx, lp, s)
+    _check(O_, Q, K, V, idx, lp, H, N, bk)
+
+
+def test_attn_tiny_config_identical_oracle_plan():
+    w = WORKLOADS["tiny"]
+    Q, K, V = make_qkv(w)
+    S = np.stack([O.select_head(np64(Q[0, h]), np64(K[0, h]), 128, 4, 8, 1) for h in range(w.H)])
+    idx = np.zeros((w.H, w.nQ, w.s), np.int32)
+    lp = np.zeros((w.H, w.nQ, w.s), np.float32)
+    for h in range(w.H):
+        for i in range(w.nQ):
+            idx[h, i], lp[h, i], _ = O.plan_row(S[h, i], w.s, w.philox_seed, 0, h * w.nQ + i)
+    idx_t, lp_t = torch.from_numpy(idx).reshape(-1, w.s), torch.from_numpy(lp).reshape(-1, w.s)
+    p = ab.params(w.B, w.H, w.N, w.d, w.kv_block)
+    O_ = _run(p, Q, K, V, idx_t, lp_t, w.s)
+    _check(O_, Q, K, V, idx_t, lp_t, w.H, w.N, w.kv_block)
+
+
+@pytest.mark.parametrize("N,d", [(1024, 64), (1000, 128), (300, 64)])
+def test_dense_path_equals_dense_oracle(N, d):
+    H = 2
+    Q, K, V = _qkv(H, N, d, seed=7 + N)
+    p = ab.params(1, H, N, d, kv_block=4)
+    O_ = torch.full(Q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    ab.ab_attn_dense(p, Q.cuda(), K.cuda(), V.cuda(), O_)
+    assert ab.ab_get_status() == 0
+    for h in range(H):
+        ref = O.dense_attention(np64(Q[0, h]), np64(K[0, h]), np64(V[0, h]))
+        assert_o_close(np64(O_[0, h]), ref, f"dense h{h}")
+
+
+@pytest.mark.parametrize("bk", [4, 16, 128])
+def test_all_blocks_packed_equals_dense_path_bitwise(bk):
+    """s = nK gives pi = 1 (log pi = 0) and the packed tiles are exactly the dense tiles."""
+    H, N, d = 2, 1024, 128
+    nK = N // bk
+    Q, K, V = _qkv(H, N, d, seed=3)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    idx = torch.arange(nK, dtype=torch.int32).repeat(H * 8, 1)
+    lp = torch.zeros(H * 8, nK)
+    O1 = _run(p, Q, K, V, idx, lp, nK)
+    O2 = torch.empty_like(O1)
+    ab.ab_attn_dense(p, Q.cuda(), K.cuda(), V.cuda(), O2)
+    assert ab.ab_get_status() == 0
+    assert torch.equal(O1, O2)
+
+
+def test_bad_index_status():
+    H, N, d, bk, s = 1, 256, 64, 4, 8
+    Q, K, V = _qkv(H, N, d, seed=9)
+    idx = torch.arange(s, dtype=torch.int32).repeat(2, 1)
+    idx[1, 3] = 10_000
+    lp = torch.zeros(2, s)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    O_ = torch.empty(Q.shape, dtype=torch.bfloat16, device="cuda")
+    ab.ab_attn(p, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), lp.cuda(), s, O_)
+    assert ab.ab_get_status() == -7
+    assert ab.ab_get_status() == 0  # cleared
+    # the masked block is simply absent: query block 1 attends to the 7 valid blocks
+    keep = [0, 1, 2, 4, 5, 6, 7]
+    ref = O.attn_block(np64(Q[0, 0, 128:]), np64(K[0, 0]), np64(V[0, 0]), keep, [0.0] * 7, bk)
+    assert_o_close(np64(O_[0, 0, 128:]), ref)

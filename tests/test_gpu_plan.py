@@ -1,0 +1,127 @@
+"""GPU parity of the SIP planner (ab_plan, ab_sample) against the CPU oracle.
+
+Sample indices must be bit-exact; log-probabilities may differ by at most one fp32
+ulp (the fp64 logarithm is rounded to fp32 on both sides, and CUDA's and the host's
+fp64 log may differ in the last fp64 bit).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_ibcs_b200 as ab
+from block_sparse_attention_ibcs_b200.inputs import WORKLOADS, make_qkv, random_scores
+from oracle import abattn_oracle as O
+
+from _util import f32_ulp_diff, np64
+
+pytestmark = pytest.mark.gpu
+
+TWO32 = 1 << 32
+
+
+def _gpu_plan(p, S, s, seed, offset, fn=ab.ab_plan):
+    rows = S.shape[0] * S.shape[1] * S.shape[2] if S.dim() == 4 else S.shape[0]
+    idx = torch.full((rows, s), -7, dtype=torch.int32, device="cuda")
+    lp = torch.full((rows, s), 99.0, dtype=torch.float32, device="cuda")
+    fn(p, S.contiguous(), s, seed, offset, idx, lp)
+    assert ab.ab_get_status() == 0
+    return idx.cpu().numpy(), lp.cpu().numpy()
+
+
+def _check_rows(S_cpu, idx, lp, s, seed, offset, rows):
+    for r in rows:
+        ridx, rlp, qp = O.plan_row(S_cpu[r], s, seed, offset, r)
+        assert np.array_equal(idx[r], ridx), f"row {r}: idx differs"
+        assert f32_ulp_diff(lp[r], rlp).max() <= 1, f"row {r}: logpi differs"
+        assert int(qp.sum()) == s * TWO32
+
+
+def test_plan_tiny_config_from_oracle_scores():
+    w = WORKLOADS["tiny"]
+    Q, K, _ = make_qkv(w)
+    S = np.stack([O.select_head(np64(Q[0, h]), np64(K[0, h]), 128, w.kv_block, 8, 1)
+                  for h in range(w.H)])  # [H, nQ, nK] fp32
+    p = ab.params(w.B, w.H, w.N, w.d, w.kv_block)
+    St = torch.from_numpy(S).cuda().reshape(1, w.H, w.nQ, w.nK)
+    for s in (32, 1, 255, 256):
+        idx, lp = _gpu_plan(p, St, s, w.philox_seed, 0)
+        _check_rows(S.reshape(-1, w.nK), idx, lp, s, w.philox_seed, 0, range(w.H * w.nQ))
+    # s = all blocks: pi = 1 everywhere
+    idx, lp = _gpu_plan(p, St, 256, 5, 3)
+    assert (idx == np.arange(256)).all() and (lp == 0).all()
+
+
+@pytest.mark.parametrize("name", ["wan13b", "hunyuan13b"])
+def test_plan_full_shape_random_scores(name):
+    w = WORKLOADS[name]
+    rows = w.B * w.H * w.nQ
+    S = random_scores(rows, w.nK, seed=11, device="cuda")
+    p = ab.params(w.B, w.H, w.N, w.d, w.kv_block)
+    idx, lp = _gpu_plan(p, S, w.s, w.philox_seed, 7)
+    # every row: exactly s distinct ascending in-range indices (cheap host invariants)
+    assert (np.diff(idx, axis=1) > 0).all() and idx.min() >= 0 and idx.max() < w.nK
+    assert (lp <= 0).all()
+    pick = [0, 1, w.nQ - 1, rows // 2, rows - 1] + list(np.random.default_rng(0).integers(0, rows, 11))
+    S_cpu = S[torch.tensor(pick, device="cuda")].cpu().numpy()
+    for k, r in enumerate(pick):
+        ridx, rlp, _ = O.plan_row(S_cpu[k], w.s, w.philox_seed, 7, int(r))
+        assert np.array_equal(idx[r], ridx), f"row {r}"
+        assert f32_ulp_diff(lp[r], rlp).max() <= 1
+
+
+def test_plan_edge_rows():
+    nK = 256
+    rows = []
+    rng = np.random.default_rng(3)
+    x = np.exp(2 * rng.standard_normal(nK)); rows.append(x / x.sum())        # ordinary
+    z = np.zeros(nK); z[[5, 9, 200]] = [0.5, 0.3, 0.2]; rows.append(z)        # fewer than s positive
+    o = np.full(nK, 1e-9); o[17] = 1.0; rows.append(o / o.sum())              # one dominant block
+    u = np.full(nK, 1.0 / nK); rows.append(u)                                 # uniform
+    t = np.exp(6 * rng.standard_normal(nK)); rows.append(t / t.sum())         # very heavy tail
+    n = x / x.sum(); n = n.copy(); n[[3, 4]] = np.nan; n[7] = -1.0; rows.append(n)  # NaN / negative
+    e = np.zeros(nK); rows.append(e)                                          # all zero
+    d = np.exp(rng.standard_normal(nK)); d[100:] = 0; rows.append(d / d.sum())  # zero tail
+    S = np.stack(rows).astype(np.float32)
+    R = len(rows)
+    assert R == 8  # N = 1024 tokens: 8 query blocks x 256 KV blocks of 4
+    p = ab.params(1, 1, 1024, 64, kv_block=4)
+    for s in (1, 8, 32, 255):
+        idx, lp = _gpu_plan(p, torch.from_numpy(S).cuda(), s, 123, 456)
+        _check_rows(S, idx, lp, s, 123, 456, range(R))
+
+
+def test_sample_given_oracle_pi_bit_exact():
+    rng = np.random.default_rng(4)
+    nK, R, s = 256, 8, 24
+    S = rng.dirichlet(np.full(nK, 0.3), size=R).astype(np.float32)
+    pi = np.stack([(O.inclusion_fixed_point(S[r], s)[0].astype(np.float64) / TWO32) for r in range(R)])
+    pi = pi.astype(np.float32)
+    p = ab.params(1, 1, 128 * R, 64, kv_block=4)
+    assert -(-128 * R // 4) == nK
+    idx, lp = _gpu_plan(p, torch.from_numpy(pi).cuda(), s, 9, 1, fn=ab.ab_sample)
+    for r in range(R):
+        ridx, rlp, qp = O.sample_row(pi[r], s, 9, 1, r)
+        assert np.array_equal(idx[r], ridx)
+        assert f32_ulp_diff(lp[r], rlp).max() <= 1
+        # the draw reproduces the given probabilities to fp32 resolution (the fixed-point
+        # cap may move about s * 2^-23 of mass off the last non-saturated block)
+        assert np.allclose(qp.astype(np.float64) / TWO32, pi[r], rtol=2e-6, atol=s * 2.0 ** -22)
+
+
+def test_sample_monte_carlo_inclusion_frequencies():
+    """Over many offsets the GPU's inclusion frequencies match pi (same rows, new U)."""
+    rng = np.random.default_rng(5)
+    nK, s = 256, 20
+    x = np.exp(1.5 * rng.standard_normal(nK))
+    S = (x / x.sum()).astype(np.float32)
+    R = 2048  # rows = independent draws (the row index enters the Philox counter)
+    p = ab.params(1, R // 8, 1024, 64, kv_block=4)  # 256 heads x 8 query blocks, nK = 256
+    St = torch.from_numpy(np.tile(S, (R, 1))).cuda()
+    idx, _ = _gpu_plan(p, St, s, 77, 0)
+    hits = np.bincount(idx.ravel(), minlength=nK) / R
+    qp, _, _ = O.inclusion_fixed_point(S, s)
+    pi = qp.astype(np.float64) / TWO32
+    se = np.sqrt(np.maximum(pi * (1 - pi), 1e-12) / R)
+    assert np.abs((hits - pi) / se)[(pi > 0) & (pi < 1)].max() < 5.5
+    assert (hits[pi == 1] == 1).all()
