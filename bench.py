@@ -126,15 +126,31 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host scalar over all ranks (NCCL on the GPU, gloo on the CPU)."""
     import torch
 
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w, rank):
+    """Weak scaling: rank r processes its own independent layer (same shape, own seed)."""
+    import dataclasses
+
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank, philox_seed=w.philox_seed + 1000 * rank)
+
+
+def shard_heads(H, world, rank):
+    """Head-parallel split of one layer: contiguous head range of this rank."""
+    base, extra = divmod(H, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
 
 
 def kept_flops(w):
@@ -160,9 +176,7 @@ def run_ours(args, world, rank, local):
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     # each rank runs an independent layer (different seed): weak scaling
-    import dataclasses
-
-    w_r = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    w_r = rank_workload(w, rank)
     Q, K, V = make_qkv(w_r, device=dev)
     reuse = max(1, w.plan_reuse)
     pert = []
@@ -186,14 +200,21 @@ def run_ours(args, world, rank, local):
     def E():
         return torch.cuda.Event(enable_timing=True)
 
+    only_attn = args.only == "attn"
+    if only_attn:  # one plan, made before timing; the step is the attention calls alone
+        ab.ab_select(p, Q, K, S, ws)
+        ab.ab_plan(p, S, w.s, w.philox_seed, 0, idx, lp)
+
     def step(i, record):
         if record:
             e0, e1, e2 = E(), E(), E()
             e0.record(stream)
-        ab.ab_select(p, Q, K, S, ws)
+        if not only_attn:
+            ab.ab_select(p, Q, K, S, ws)
         if record:
             e1.record(stream)
-        ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
+        if not only_attn:
+            ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
         if record:
             e2.record(stream)
         att = []
@@ -242,7 +263,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not only_attn:
         e2e = run_e2e(args, w, p, Q, K, pert, reuse, world, dev)
 
     peak_t = peaks["bf16_tflops_sustained"]
@@ -267,7 +288,7 @@ def run_ours(args, world, rank, local):
                      "frac": round(attn_tflops / peak_t, 4),
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
                      "traffic": args.traffic},
-        "gpu_launches": args.steps * (4 + 1 + reuse),
+        "gpu_launches": args.steps * ((0 if only_attn else 4 + 1) + reuse),
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -341,8 +362,9 @@ def cpu_baseline(w, seconds=15.0):
     Kp = O.pool_keys(k, w.kv_block)
     done = 0
     rows_done = 0
-    qbs = list(range(0, w.nQ, max(1, w.nQ // 64)))
+    qbs = np.random.default_rng(0).permutation(w.nQ)  # fixed order; stops at the time budget
     for i in qbs:
+        i = int(i)
         Qb = q[i * 128: min(w.N, (i + 1) * 128)]
         cent, wt, _, _ = O.kmeans_block(Qb, w.clusters, w.kmeans_iters)
         S = O.block_scores(cent, wt, Kp).astype(np.float32)
@@ -393,6 +415,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b")
+    ap.add_argument("--only", default="all", choices=["all", "attn"],
+                    help="attn: time only the attention calls (for kernel profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -258,13 +258,16 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 128; ++c) mt = fmaxf(mt, z[c]);
+      // Lazy rescale, decided per warp: tcgen05.ld/st are warp-collective, so when any
+      // row of the warp has to raise its reference max, every row of the warp moves to
+      // max(m_run, mt) (alpha = 1 where nothing changes) and the warp rescales O.
+      const bool need = mt > m_run + LAZY_RESCALE_LOG2;  // always true on a row's first finite tile
+      const bool rescale = __any_sync(0xffffffffu, need);
       float alpha = 1.f;
-      bool rescale = false;
-      if (mt > m_run + LAZY_RESCALE_LOG2 || m_run == -INFINITY) {
+      if (rescale) {
         const float m_new = fmaxf(mt, m_run);
         if (m_new != -INFINITY) {
           alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
-          rescale = (m_run != -INFINITY);
           m_run = m_new;
         }
       }
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
-      if (rescale) {
+      if (rescale && t > 0) {  // warp-uniform; O holds no data before PV(0)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t v[32];

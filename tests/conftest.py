@@ -9,3 +9,4 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workload")
+    config.addinivalue_line("markers", "timeout: per-test time limit (pytest-timeout)")
