@@ -52,18 +52,20 @@ struct AttnSmem {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + TILE_BYTES;        // 2 stages
   static constexpr uint32_t V_OFF = K_OFF + 2 * TILE_BYTES;    // 2 stages
-  static constexpr uint32_t P_OFF = V_OFF + 2 * TILE_BYTES;    // 128 x 128 bf16
-  static constexpr uint32_t BIAS_OFF = P_OFF + 128u * 128u * 2u;  // 2 x 128 fp32
+  static constexpr uint32_t P_BYTES = 128u * 128u * 2u;       // 128 x 128 bf16
+  static constexpr uint32_t P_OFF = V_OFF + 2 * TILE_BYTES;    // 2 buffers
+  static constexpr uint32_t BIAS_OFF = P_OFF + 2 * P_BYTES;    // 2 x 128 fp32
   static constexpr uint32_t BAR_OFF = BIAS_OFF + 2u * 128u * 4u;
-  static constexpr uint32_t NBARS = 12;
+  static constexpr uint32_t NBARS = 14;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBARS * 8u;
   static constexpr uint32_t BYTES = MISC_OFF + 16u;
   static constexpr uint32_t ALLOC = BYTES + 1024u;  // slack for 1024-byte alignment
+  static_assert(ALLOC <= 232448u, "exceeds the 227 KB shared-memory limit per block");
 };
 
-// barrier slots
-enum { B_QFULL = 0, B_FULL0 = 1, B_EMPTY0 = 3, B_SFULL0 = 5, B_SFREE0 = 7, B_PFULL = 9,
-       B_PVDONE = 10, B_DRAIN = 11 };
+// barrier slots (pairs are indexed by tile parity)
+enum { B_QFULL = 0, B_FULL0 = 1, B_EMPTY0 = 3, B_SFULL0 = 5, B_SFREE0 = 7, B_PFULL0 = 9,
+       B_PVDONE0 = 11, B_DRAIN = 13 };
 
 template <int D, bool DENSE>
 __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
@@ -94,9 +96,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       mbar_init(&bars[B_EMPTY0 + b], 1);
       mbar_init(&bars[B_SFULL0 + b], 1);
       mbar_init(&bars[B_SFREE0 + b], 128);
+      mbar_init(&bars[B_PFULL0 + b], 128);
+      mbar_init(&bars[B_PVDONE0 + b], 1);
     }
-    mbar_init(&bars[B_PFULL], 128);
-    mbar_init(&bars[B_PVDONE], 1);
     mbar_init(&bars[B_DRAIN], 1);
     fence_mbar_init();
   }
@@ -116,9 +118,35 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     // ================================================================ producers
     const int p = tid - 128;       // 0..127
     const int u = p & 15;          // 16-byte unit within a 256-byte (D=128) row
-    const int rsub = p >> 4;       // 0..7
+    const int rsub = p >> 4;       // 0..7: this thread copies rows rsub, rsub+8, ...
     constexpr int UNITS = D / 8;   // 16-byte units per row
     const size_t plan_off = (size_t)blockIdx.x * a.s;
+    const int nb = 128 >> a.bk_shift;  // sampled blocks per tile
+
+    // Plan entries of one tile, spread over the warp: lane e (+32k) holds the tile's
+    // block e -- its index (-1 for padding or a rejected entry) and log pi.  Loaded
+    // coalesced one tile ahead and broadcast to the copying lanes with shuffles.
+    int jc[4], jn[4];
+    float lc[4], ln[4];
+    auto fetch = [&](int t, int (&jr)[4], float (&lr)[4]) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = lane + 32 * k;
+        const int m = t * nb + e;
+        jr[k] = -1;
+        lr[k] = 0.f;
+        if (!DENSE && e < nb && m < a.s) {
+          const int j = __ldg(a.idx + plan_off + m);
+          if (j < 0 || j >= a.nK) {
+            ab_flag(AB_ERR_DEVICE_CHECK);
+          } else {
+            jr[k] = j;
+            lr[k] = __ldg(a.logpi + plan_off + m);
+          }
+        }
+      }
+    };
+    if (!DENSE) fetch(0, jc, lc);
 
     // Q tile: rows row0..row0+127 (zero beyond N)
     for (int r = rsub; r < 128; r += 8) {
@@ -133,36 +161,38 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
 
     for (int t = 0; t < T; ++t) {
       const int st = t & 1;
+      if (!DENSE && t + 1 < T) fetch(t + 1, jn, ln);  // in flight while this tile is issued
       if (t >= 2 && !mbar_wait(&bars[B_EMPTY0 + st], ((t >> 1) - 1) & 1, abort_flag, a.timeout_ns))
         break;
       const uint32_t kdst = sbase + L::K_OFF + st * L::TILE_BYTES;
       const uint32_t vdst = sbase + L::V_OFF + st * L::TILE_BYTES;
-      for (int r = rsub; r < 128; r += 8) {
-        const int pos = t * 128 + r;  // position in the packed token sequence
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int r = rsub + 8 * i;  // row of the tile (= column of S)
         int tok;
         float b2;
         bool ok;
         if (DENSE) {
-          tok = pos;
+          tok = t * 128 + r;
           ok = tok < a.N;
           b2 = 0.f;
         } else {
-          const int m = pos >> a.bk_shift;
-          const int within = pos & (a.bk - 1);
-          ok = m < a.s;
-          int j = 0;
-          b2 = 0.f;
-          if (ok) {
-            j = __ldg(a.idx + plan_off + m);
-            if (j < 0 || j >= a.nK) {
-              if (u == 0) ab_flag(AB_ERR_DEVICE_CHECK);
-              ok = false;
-            } else {
-              b2 = -__ldg(a.logpi + plan_off + m) * LOG2E;
+          const int ml = r >> a.bk_shift;  // block of the tile holding this row
+          const int src = ml & 31;
+          int j = __shfl_sync(0xffffffffu, jc[0], src);
+          float lp = __shfl_sync(0xffffffffu, lc[0], src);
+          if (nb > 32) {  // warp-uniform: more than 32 blocks per tile (kv_block < 4)
+            const int reg = ml >> 5;
+#pragma unroll
+            for (int k = 1; k < 4; ++k) {
+              const int jk = __shfl_sync(0xffffffffu, jc[k], src);
+              const float lk = __shfl_sync(0xffffffffu, lc[k], src);
+              if (reg == k) { j = jk; lp = lk; }
             }
           }
-          tok = j * a.bk + within;
-          ok = ok && tok < a.N;
+          tok = j * a.bk + (r & (a.bk - 1));
+          ok = j >= 0 && tok < a.N;
+          b2 = -lp * LOG2E;
         }
         if (u < UNITS) {
           const size_t goff = head_off + (size_t)(ok ? tok : 0) * D + u * 8;
@@ -171,6 +201,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           cp_async_16(vdst + soff, a.V + goff, ok ? 16u : 0u);
         }
         if (u == 0) bias[st * 128 + r] = ok ? b2 : -INFINITY;
+      }
+      if (!DENSE) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { jc[k] = jn[k]; lc[k] = ln[k]; }
       }
       if (a.debug_skip_arrive && t == 0) continue;  // test knob: never signal tile 0
       mbar_arrive(&bars[B_FULL0 + st]);
@@ -185,17 +219,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       bool ok = mbar_wait(&bars[B_QFULL], 0, abort_flag, a.timeout_ns);
       // issue PV for tile tp (P ready, V in stage tp&1)
       auto issue_pv = [&](int tp) -> bool {
-        if (!mbar_wait(&bars[B_PFULL], tp & 1, abort_flag, a.timeout_ns)) return false;
+        if (!mbar_wait(&bars[B_PFULL0 + (tp & 1)], (tp >> 1) & 1, abort_flag, a.timeout_ns))
+          return false;
         tc_fence_after();
         const uint32_t vbase = sbase + L::V_OFF + (tp & 1) * L::TILE_BYTES;
-        const uint32_t pbase = sbase + L::P_OFF;
+        const uint32_t pbase = sbase + L::P_OFF + (tp & 1) * L::P_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
           const uint64_t ad = sdesc_sw128(pbase + (kk >> 2) * L::CHUNK_BYTES + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(vbase + kk * 2048, L::CHUNK_BYTES, 1024);
           umma_f16_ss(TM_O, ad, bd, IDESC_PV, (tp > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars[B_PVDONE]);
+        umma_commit(&bars[B_PVDONE0 + (tp & 1)]);
         umma_commit(&bars[B_EMPTY0 + (tp & 1)]);
         return true;
       };
@@ -233,7 +268,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_run = -INFINITY;  // reference max (log2 domain)
     float l_run = 0.f;
-    uint8_t* prow = smem + L::P_OFF;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int st = t & 1;
@@ -251,7 +285,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         tmem_ld_32x32b_x32(sadr + c0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) z[c0 + c] = fmaf(__uint_as_float(v[c]), a.scale_log2, bcol[c0 + c]);
+        for (int c = 0; c < 32; c += 4) {
+          const float4 b4 = *(const float4*)(bcol + c0 + c);
+          z[c0 + c] = fmaf(__uint_as_float(v[c]), a.scale_log2, b4.x);
+          z[c0 + c + 1] = fmaf(__uint_as_float(v[c + 1]), a.scale_log2, b4.y);
+          z[c0 + c + 2] = fmaf(__uint_as_float(v[c + 2]), a.scale_log2, b4.z);
+          z[c0 + c + 3] = fmaf(__uint_as_float(v[c + 3]), a.scale_log2, b4.w);
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars[B_SFREE0 + st]);
@@ -272,23 +312,32 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         }
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+      // P buffer st is free once PV(t-2) has completed
+      if (t >= 2) {
+        ok = mbar_wait(&bars[B_PVDONE0 + st], ((t >> 1) - 1) & 1, abort_flag, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      }
+      uint8_t* prow = smem + L::P_OFF + st * L::P_BYTES;
       float lsum = 0.f;
-      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = fast_exp2(z[c] - mref);
-        const float p1 = fast_exp2(z[c + 1] - mref);
-        lsum += p0 + p1;
-        pk[c >> 1] = pack_bf16x2_rn(p0, p1);
+      for (int uu = 0; uu < 16; ++uu) {  // 8 keys per 16-byte unit of P
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = fast_exp2(z[8 * uu + 2 * e] - mref);
+          const float p1 = fast_exp2(z[8 * uu + 2 * e + 1] - mref);
+          lsum += p0 + p1;
+          pk[e] = pack_bf16x2_rn(p0, p1);
+        }
+        const uint32_t off = (uu >> 3) * 16384u + sw128_off(r, uu & 7);
+        *(uint4*)(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       l_run = l_run * alpha + lsum;
-      // P buffer and O are free once PV(t-1) has completed
-      if (t >= 1) {
-        ok = mbar_wait(&bars[B_PVDONE], (t - 1) & 1, abort_flag, a.timeout_ns);
+      if (rescale && t > 0) {  // warp-uniform; O holds no data before PV(0)
+        // O is stable once PV(t-1) has completed
+        ok = mbar_wait(&bars[B_PVDONE0 + (st ^ 1)], ((t - 1) >> 1) & 1, abort_flag, a.timeout_ns);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-      }
-      if (rescale && t > 0) {  // warp-uniform; O holds no data before PV(0)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t v[32];
@@ -300,16 +349,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         }
         tmem_wait_st();
       }
-#pragma unroll
-      for (int uu = 0; uu < 16; ++uu) {  // 8 keys per 16-byte unit
-        const uint32_t off = (uu >> 3) * 16384u + sw128_off(r, uu & 7);
-        *(uint4*)(prow + off) = make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
-      }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL]);
+      mbar_arrive(&bars[B_PFULL0 + st]);
     }
-    if (ok && T > 0) ok = mbar_wait(&bars[B_PVDONE], (T - 1) & 1, abort_flag, a.timeout_ns);
+    if (ok && T > 0)
+      ok = mbar_wait(&bars[B_PVDONE0 + ((T - 1) & 1)], ((T - 1) >> 1) & 1, abort_flag, a.timeout_ns);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
