@@ -174,3 +174,18 @@ def ab_attn_dense(p, Q, K, V, O, stream=None):
 def ab_get_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return lib().ab_get_status(_stream(stream))
+
+
+def ab_select_noalloc(p, Q, K, S, stream=None):
+    """ab_select without a workspace: the library's built-in scratch (16 MiB per GPU) is used.
+
+    For callers that may not allocate device memory and have no scratch buffer to pass.
+    Calls that overlap on the GPU share that scratch and race; serialise them.
+    """
+    import torch
+
+    f = lib().ab_select_noalloc
+    f.argtypes = [_P, _vp, _vp, _vp, _vp]
+    f.restype = ctypes.c_int
+    _check(f(ctypes.byref(p), _ptr(Q, "Q", torch.bfloat16), _ptr(K, "K", torch.bfloat16),
+             _ptr(S, "S", torch.float32), _stream(stream)), "ab_select_noalloc")

@@ -304,3 +304,77 @@ const char* ab_status_string(ab_status s) {
 int ab_version(void) { return 100; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// ab_select_noalloc: the selector with its scratch compiled into the library.
+//
+// Some callers cannot give this library a workspace: a plugin inside a host framework
+// that owns all device memory and exposes no scratch allocator to its plugins, or a
+// serving loop whose device-memory plan is frozen at start-up and which must not call
+// cudaMalloc/cudaFree (they synchronise the device and stall every stream) while
+// requests are in flight.  For those callers the selector's scratch -- pooled keys,
+// centroids, shares and per-centroid softmax statistics -- lives in one fixed array
+// below instead of a caller buffer.
+// ------------------------------------------------------------------------------------
+
+#include <mutex>
+
+// Capacity of the built-in scratch.  Every GPU that loads the library holds this much
+// device memory until the process exits.
+#define AB_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+static __device__ __align__(256) uint8_t g_ab_noalloc_scratch[AB_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The host-side symbol is
+// only a stand-in, so the address is looked up once per device (with that device
+// current) and cached.
+ab_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status();
+  if (dev < 0 || dev >= kMaxDevices) return AB_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_ab_noalloc_scratch);
+    if (e != cudaSuccess || addr == nullptr) {
+      fprintf(stderr, "abattn: cannot resolve the built-in scratch on device %d: %s\n", dev,
+              cudaGetErrorString(e));
+      cudaGetLastError();
+      return AB_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return AB_OK;
+}
+
+}  // namespace
+
+extern "C" ab_status ab_select_noalloc(const ab_params* p, const void* Q, const void* K, float* S,
+                                       void* stream) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(S)) return AB_ERR_INVALID_ARG;
+  const size_t need = carve(d, nullptr).bytes;
+  if (need > AB_NOALLOC_SCRATCH_BYTES) {
+    fprintf(stderr,
+            "abattn: ab_select_noalloc needs %zu bytes of scratch for this shape but the built-in "
+            "array holds %u; call ab_select with a workspace instead\n",
+            need, (unsigned)AB_NOALLOC_SCRATCH_BYTES);
+    return AB_ERR_WORKSPACE;
+  }
+  void* base = nullptr;
+  r = noalloc_scratch(&base);
+  if (r != AB_OK) return r;
+  const Workspace ws = carve(d, base);
+  cudaStream_t st = (cudaStream_t)stream;
+  return (d.d == 128) ? run_select<128>(d, Q, K, S, ws, nullptr, st)
+                      : run_select<64>(d, Q, K, S, ws, nullptr, st);
+}

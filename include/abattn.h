@@ -141,6 +141,29 @@ const char* ab_status_string(ab_status s);
 /* Library version, major*10000 + minor*100 + patch. */
 int ab_version(void);
 
+/* ab_select for callers that cannot provide a workspace.  The paper has no counterpart:
+ * this is a packaging variant of ab_select, same inputs, same S.
+ *
+ * Who needs it: code that may not allocate device memory and has no scratch buffer to
+ * pass -- e.g. a plugin whose host framework owns every device allocation and gives its
+ * plugins no scratch allocator, or a serving loop whose memory plan is fixed at start-up
+ * and must not call cudaMalloc/cudaFree (they synchronise the device) mid-flight.
+ *
+ * Instead of `ws`, the call uses one scratch array compiled into the library
+ * (16 MiB per GPU, held from library load until process exit).  It allocates nothing
+ * itself.  Shapes whose ab_workspace_bytes exceeds 16 MiB (about two Wan2.1 heads of
+ * N = 75,600 at d = 128) are rejected with AB_ERR_WORKSPACE and a message on stderr;
+ * use ab_select for them.
+ *  - The first call on each device looks up the array's device address (with that device
+ *    current) and caches it; make that first call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the previous call's contents
+ *    (every byte the selector reads is written earlier in the same call, so nothing has
+ *    to be cleared).  Calls whose work overlaps on the GPU -- on different streams, or
+ *    from different threads -- race on the array: serialise them.
+ * Other arguments, errors and results are those of ab_select.                         */
+ab_status ab_select_noalloc(const ab_params* p, const void* Q, const void* K, float* S,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif
