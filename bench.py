@@ -201,7 +201,10 @@ def run_ours(args, world, rank, local):
         return torch.cuda.Event(enable_timing=True)
 
     only_attn = args.only == "attn"
-    if only_attn:  # one plan, made before timing; the step is the attention calls alone
+    run_select = args.only in ("all", "select")
+    run_plan = args.only in ("all", "plan")
+    run_attn = args.only in ("all", "attn")
+    if args.only != "all":  # stage-only runs (kernel profiling): make the inputs once
         ab.ab_select(p, Q, K, S, ws)
         ab.ab_plan(p, S, w.s, w.philox_seed, 0, idx, lp)
 
@@ -209,16 +212,16 @@ def run_ours(args, world, rank, local):
         if record:
             e0, e1, e2 = E(), E(), E()
             e0.record(stream)
-        if not only_attn:
+        if run_select:
             ab.ab_select(p, Q, K, S, ws)
         if record:
             e1.record(stream)
-        if not only_attn:
+        if run_plan:
             ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
         if record:
             e2.record(stream)
         att = []
-        for c in range(reuse):
+        for c in range(reuse if run_attn else 0):
             qa, ka, va = pert[c]
             if record:
                 a0, a1 = E(), E()
@@ -254,7 +257,8 @@ def run_ours(args, world, rank, local):
     ms_step = ms_total / args.steps
     sel_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, e2, _ in ev["steps"])
     plan_ms = statistics.mean(e1.elapsed_time(e2) for e0, e1, e2, _ in ev["steps"])
-    attn_ms = statistics.mean(a0.elapsed_time(a1) for *_, att in ev["steps"] for a0, a1 in att)
+    attn_ms = (statistics.mean(a0.elapsed_time(a1) for *_, att in ev["steps"] for a0, a1 in att)
+               if run_attn else float("nan"))
     F = kept_flops(w)
     value = world * reuse * F / (ms_step * 1e-3) / 1e12
     attn_tflops = F / (attn_ms * 1e-3) / 1e12
@@ -263,7 +267,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API from pinned host buffers
     e2e = None
-    if not args.no_e2e and not only_attn:
+    if not args.no_e2e and args.only == "all":
         e2e = run_e2e(args, w, p, Q, K, pert, reuse, world, dev)
 
     peak_t = peaks["bf16_tflops_sustained"]
@@ -288,7 +292,7 @@ def run_ours(args, world, rank, local):
                      "frac": round(attn_tflops / peak_t, 4),
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
                      "traffic": args.traffic},
-        "gpu_launches": args.steps * ((0 if only_attn else 4 + 1) + reuse),
+        "gpu_launches": args.steps * (4 * run_select + run_plan + reuse * run_attn),
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -382,6 +386,83 @@ def cpu_baseline(w, seconds=15.0):
             "ms_per_query_block": round(1e3 * dt / done, 1)}
 
 
+def run_sweep(args):
+    """Granularity sweep at the Wan2.1-1.3B shape (not a bench line; prints one JSON line).
+
+    For KV block 4, 16, 64, 128 at a fixed budget of 8192 kept tokens per query block:
+    packed tiles per query block (ceil(s*bk/128) = 64 in every case) against one tile
+    per selected block (s), select/plan/attention times, and the relative L2 error of
+    the sparse output against the fp64 dense oracle on head 0 (32 fixed query blocks
+    including the last).  Also times s = all blocks through the packed kernel against the
+    same kernel's dense path.
+    """
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_ibcs_b200 as ab
+    from block_sparse_attention_ibcs_b200.inputs import WORKLOADS, make_qkv
+    from oracle import abattn_oracle as O
+
+    torch.cuda.set_device(0)
+    base = WORKLOADS["sweep_bk4"]
+    Q, K, V = make_qkv(base, device="cuda")
+    qb_list = sorted(set(np.linspace(0, base.nQ - 1, 32).astype(int).tolist()))
+    rows = np.concatenate([np.arange(i * 128, min(base.N, (i + 1) * 128)) for i in qb_list])
+    q0, k0, v0 = (t[0, 0].double().cpu().numpy() for t in (Q, K, V))
+    dense_ref = O.dense_attention(q0[rows], k0, v0)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps=3):
+        fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    out = {"workload": "Wan2.1-1.3B shape: B=1 H=12 N=75600 d=128, 8192 kept tokens per query block",
+           "dense_reference": "fp64 oracle, head 0, query blocks " + ",".join(map(str, qb_list)),
+           "cases": []}
+    for bk in (4, 16, 64, 128):
+        w = WORKLOADS[f"sweep_bk{bk}"]
+        p = ab.params(w.B, w.H, w.N, w.d, bk)
+        R = w.B * w.H * w.nQ
+        S = torch.empty(w.B, w.H, w.nQ, w.nK, device="cuda")
+        ws = torch.empty(ab.ab_workspace_bytes(p), dtype=torch.uint8, device="cuda")
+        idx = torch.empty(R, w.s, dtype=torch.int32, device="cuda")
+        lp = torch.empty(R, w.s, device="cuda")
+        Od = torch.empty_like(Q)
+        t_sel = timed(lambda: ab.ab_select(p, Q, K, S, ws))
+        t_plan = timed(lambda: ab.ab_plan(p, S, w.s, w.philox_seed, 0, idx, lp))
+        t_attn = timed(lambda: ab.ab_attn(p, Q, K, V, idx, lp, w.s, Od))
+        assert ab.ab_get_status() == 0
+        got = Od[0, 0].double().cpu().numpy()[rows]
+        rel = float(np.linalg.norm(got - dense_ref) / np.linalg.norm(dense_ref))
+        out["cases"].append({"kv_block": bk, "s": w.s, "nK": w.nK,
+                             "tiles_per_query_block_packed": -(-w.s * bk // 128),
+                             "tiles_per_query_block_one_per_block": w.s,
+                             "select_ms": round(t_sel, 3), "plan_ms": round(t_plan, 3),
+                             "attn_ms": round(t_attn, 3),
+                             "attn_tflops": round(kept_flops(w) / (t_attn * 1e-3) / 1e12, 1),
+                             "rel_l2_vs_dense_fp64": round(rel, 5)})
+    # s = all blocks through the packed kernel vs the dense path (bk = 128: 591 blocks)
+    w = WORKLOADS["sweep_bk128"]
+    p = ab.params(w.B, w.H, w.N, w.d, 128)
+    R = w.B * w.H * w.nQ
+    idx = torch.arange(w.nK, dtype=torch.int32, device="cuda").repeat(R, 1).contiguous()
+    lp = torch.zeros(R, w.nK, device="cuda")
+    O1, O2 = torch.empty_like(Q), torch.empty_like(Q)
+    t_pk = timed(lambda: ab.ab_attn(p, Q, K, V, idx, lp, w.nK, O1), reps=2)
+    t_dn = timed(lambda: ab.ab_attn_dense(p, Q, K, V, O2), reps=2)
+    dense_flops = 4.0 * w.B * w.H * w.N * w.N * w.d
+    out["all_blocks"] = {"packed_ms": round(t_pk, 3), "dense_path_ms": round(t_dn, 3),
+                         "dense_tflops": round(dense_flops / (t_dn * 1e-3) / 1e12, 1),
+                         "bitwise_equal": bool(torch.equal(O1, O2))}
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args, world, rank):
     """The reference arm: the CPU oracle (the pages publish no implementation)."""
     if rank != 0:
@@ -415,8 +496,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b")
-    ap.add_argument("--only", default="all", choices=["all", "attn"],
-                    help="attn: time only the attention calls (for kernel profiling)")
+    ap.add_argument("--only", default="all", choices=["all", "attn", "select", "plan"],
+                    help="time one stage only (kernel profiling); the step is then that stage")
+    ap.add_argument("--sweep", action="store_true",
+                    help="granularity sweep (KV block 4..128) at the Wan2.1-1.3B shape")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -425,6 +508,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -59,6 +59,7 @@ _SIGS = {
     "ab_sample": [_P, _vp, _i, _u64, _u64, _vp, _vp, _vp],
     "ab_attn": [_P, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp],
     "ab_attn_dense": [_P, _vp, _vp, _vp, _vp, _vp],
+    "ab_attn_debug": [_P, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _u64, _vp, _vp],
     "ab_get_status": [_vp],
     "ab_status_string": [_i],
     "ab_version": [],
@@ -169,6 +170,19 @@ def ab_attn_dense(p, Q, K, V, O, stream=None):
     bf = torch.bfloat16
     _check(lib().ab_attn_dense(ctypes.byref(p), _ptr(Q, "Q", bf), _ptr(K, "K", bf), _ptr(V, "V", bf),
                                _ptr(O, "O", bf), _stream(stream)), "ab_attn_dense")
+
+
+def ab_attn_debug(p, Q, K, V, idx, logpi, s, O, skip_first_arrival, timeout_ns, trace=None,
+                  stream=None):
+    """Test/profiling hook: ab_attn with a producer arrival skipped, another device wait
+    limit, and optionally a per-tile clock64 event trace (int64 tensor of 3*16*128)."""
+    import torch
+
+    bf = torch.bfloat16
+    _check(lib().ab_attn_debug(ctypes.byref(p), _ptr(Q, "Q", bf), _ptr(K, "K", bf), _ptr(V, "V", bf),
+                               _ptr(idx, "idx", torch.int32), _ptr(logpi, "logpi", torch.float32),
+                               int(s), _ptr(O, "O", bf), int(skip_first_arrival), int(timeout_ns),
+                               _ptr(trace, "trace", torch.int64), _stream(stream)), "ab_attn_debug")
 
 
 def ab_get_status(stream=None) -> int:

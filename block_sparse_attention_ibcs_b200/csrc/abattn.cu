@@ -111,8 +111,14 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
   pool_kernel<D><<<pool_blocks, 256, 0, st>>>(a);
   kmeans_kernel<D><<<(unsigned)(d.BH * d.nQ), KM_THREADS, 0, st>>>(a);
   const unsigned sc_grid = (unsigned)(d.BH * ((d.nQ + 15) / 16));
-  score_kernel<D, 1><<<sc_grid, SC_THREADS, 0, st>>>(a);
-  score_kernel<D, 2><<<sc_grid, SC_THREADS, 0, st>>>(a);
+  using SL = ScoreSmem<D>;
+  if (cudaFuncSetAttribute(score_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SL::ALLOC) != cudaSuccess ||
+      cudaFuncSetAttribute(score_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SL::ALLOC) != cudaSuccess)
+    return launch_status();
+  score_tc_kernel<D, 1><<<sc_grid, SCT_THREADS, SL::ALLOC, st>>>(a, kDefaultTimeoutNs);
+  score_tc_kernel<D, 2><<<sc_grid, SCT_THREADS, SL::ALLOC, st>>>(a, kDefaultTimeoutNs);
   return launch_status();
 }
 
@@ -143,7 +149,7 @@ ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t
 template <int D, bool DENSE>
 ab_status run_attn(const Dims& d, const void* Q, const void* K, const void* V, const int32_t* idx,
                    const float* logpi, int s, void* O, int debug_skip, uint64_t timeout_ns,
-                   cudaStream_t st) {
+                   uint64_t* trace, cudaStream_t st) {
   AttnArgs a;
   a.Q = (const uint16_t*)Q;
   a.K = (const uint16_t*)K;
@@ -161,17 +167,26 @@ ab_status run_attn(const Dims& d, const void* Q, const void* K, const void* V, c
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   a.timeout_ns = timeout_ns;
   a.debug_skip_arrive = debug_skip;
+  a.trace = trace;
   using L = AttnSmem<D>;
-  if (cudaFuncSetAttribute(attn_kernel<D, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           L::ALLOC) != cudaSuccess)
-    return launch_status();
-  attn_kernel<D, DENSE><<<(unsigned)(d.BH * d.nQ), ATTN_THREADS, L::ALLOC, st>>>(a);
+  const unsigned grid = (unsigned)(d.BH * d.nQ);
+  if (trace) {
+    if (cudaFuncSetAttribute(attn_kernel<D, DENSE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::ALLOC) != cudaSuccess)
+      return launch_status();
+    attn_kernel<D, DENSE, true><<<grid, ATTN_THREADS, L::ALLOC, st>>>(a);
+  } else {
+    if (cudaFuncSetAttribute(attn_kernel<D, DENSE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::ALLOC) != cudaSuccess)
+      return launch_status();
+    attn_kernel<D, DENSE, false><<<grid, ATTN_THREADS, L::ALLOC, st>>>(a);
+  }
   return launch_status();
 }
 
 ab_status attn_common(const ab_params* p, const void* Q, const void* K, const void* V,
                       const int32_t* idx, const float* logpi, int s, void* O, bool dense,
-                      int debug_skip, uint64_t timeout_ns, void* stream) {
+                      int debug_skip, uint64_t timeout_ns, uint64_t* trace, void* stream) {
   Dims d;
   ab_status r = check_params(p, &d);
   if (r != AB_OK) return r;
@@ -182,10 +197,10 @@ ab_status attn_common(const ab_params* p, const void* Q, const void* K, const vo
   }
   cudaStream_t st = (cudaStream_t)stream;
   if (d.d == 128)
-    return dense ? run_attn<128, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st)
-                 : run_attn<128, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st);
-  return dense ? run_attn<64, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st)
-               : run_attn<64, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, st);
+    return dense ? run_attn<128, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, trace, st)
+                 : run_attn<128, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, trace, st);
+  return dense ? run_attn<64, true>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, trace, st)
+               : run_attn<64, false>(d, Q, K, V, idx, logpi, s, O, debug_skip, timeout_ns, trace, st);
 }
 
 ab_status select_common(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
@@ -270,12 +285,22 @@ ab_status ab_sample(const ab_params* p, const float* pi, int s, uint64_t seed, u
 
 ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* V,
                   const int32_t* idx, const float* logpi, int s, void* O, void* stream) {
-  return attn_common(p, Q, K, V, idx, logpi, s, O, false, 0, kDefaultTimeoutNs, stream);
+  return attn_common(p, Q, K, V, idx, logpi, s, O, false, 0, kDefaultTimeoutNs, nullptr, stream);
+}
+
+ab_status ab_attn_debug(const ab_params* p, const void* Q, const void* K, const void* V,
+                        const int32_t* idx, const float* logpi, int s, void* O,
+                        int skip_first_arrival, uint64_t timeout_ns, uint64_t* trace,
+                        void* stream) {
+  if (timeout_ns == 0) return AB_ERR_INVALID_ARG;
+  if (trace && ((uintptr_t)trace & 7)) return AB_ERR_INVALID_ARG;
+  return attn_common(p, Q, K, V, idx, logpi, s, O, false, skip_first_arrival ? 1 : 0, timeout_ns,
+                     trace, stream);
 }
 
 ab_status ab_attn_dense(const ab_params* p, const void* Q, const void* K, const void* V, void* O,
                         void* stream) {
-  return attn_common(p, Q, K, V, nullptr, nullptr, 0, O, true, 0, kDefaultTimeoutNs, stream);
+  return attn_common(p, Q, K, V, nullptr, nullptr, 0, O, true, 0, kDefaultTimeoutNs, nullptr, stream);
 }
 
 ab_status ab_get_status(void* stream) {

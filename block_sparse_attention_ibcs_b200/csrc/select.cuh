@@ -14,8 +14,8 @@
 //
 //   pool_kernel      Kp[bh, j, :]  = bf16(mean of block j's valid keys)
 //   kmeans_kernel    per (bh, query block): centroids (bf16) and shares (fp32)
-//   score_kernel<1>  per centroid row: running max m and sum Z of exp2(logit - m)
-//   score_kernel<2>  S[bh, i, j] = sum_c (w_c / Z_c) exp2(logit_cj - m_c)
+//   score_tc_kernel<1>  per centroid row: running max m and sum Z of exp2(logit - m)
+//   score_tc_kernel<2>  S[bh, i, j] = sum_c (w_c / Z_c) exp2(logit_cj - m_c)
 #pragma once
 
 #include "common.cuh"
@@ -24,8 +24,6 @@ namespace abattn {
 
 constexpr int CMAX = 8;          // centroid slots per query block
 constexpr int KM_THREADS = 256;
-constexpr int SC_THREADS = 128;  // 16 query blocks x 8 centroid slots
-constexpr int SC_KT = 32;        // pooled keys per shared-memory tile
 
 struct SelectArgs {
   const uint16_t* Q;
@@ -180,101 +178,229 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   if (a.labels && tid < 128) a.labels[(size_t)bh * a.nQ * 128 + row0 + tid] = (tid < n) ? lab[tid] : (int8_t)-1;
 }
 
-// ------------------------------------------------------------------ block scores (SIMT)
 
-// PASS 1: per centroid row, running (max, sum of exp2) over all pooled keys.
-// PASS 2: emit S.  CTA = 16 query blocks x 8 centroid slots = 128 rows, thread = row.
+// ------------------------------------------------------------------ block scores (tcgen05)
+//
+// The page's batched scoring ("premises & limits": query/KV blocks scored as batched
+// matrix operations) as two tensor-core streaming passes per CTA of 16 query blocks
+// (128 centroid rows), over all pooled keys of the head in tiles of 128:
+//   PASS 1: D[centroid row, key] = C Kp^T  (A = centroids, B = key tile, both K-major).
+//           Thread r (= TMEM lane r) keeps the running max m and sum Z of exp2(logit - m).
+//   PASS 2: D[key, centroid col] = Kp C^T (A = key tile, B = centroids), so thread j owns
+//           one KV block and sums (w_c / Z_c) exp2(logit - m_c) over the 8 columns of each
+//           query block in registers; S rows are stored coalesced.
+// Roles as in the attention kernel: warps 0-3 consume TMEM, warps 4-7 stream tiles with
+// cp.async (2 stages), warp 8 allocates TMEM and issues the MMAs.
+
+constexpr int SCT_THREADS = 288;
+
+template <int D>
+struct ScoreSmem {
+  static constexpr uint32_t TILE = 128u * D * 2u;
+  static constexpr uint32_t CHUNK = 128u * 128u;
+  static constexpr int STAGES = 2;
+  static constexpr uint32_t FIX_OFF = 0;  // centroid tile
+  static constexpr uint32_t KP_OFF = FIX_OFF + TILE;
+  static constexpr uint32_t COL_OFF = KP_OFF + STAGES * TILE;  // pass 2: m[128], coef[128]
+  static constexpr uint32_t BAR_OFF = COL_OFF + 2u * 128u * 4u;
+  // CFULL, FULL[2], EMPTY[2], SFULL[2], SFREE[2], DRAIN
+  static constexpr uint32_t NBARS = 10;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NBARS * 8u;
+  static constexpr uint32_t BYTES = MISC_OFF + 16u;
+  static constexpr uint32_t ALLOC = BYTES + 1024u;
+};
+
+enum { SB_CFULL = 0, SB_FULL0 = 1, SB_EMPTY0 = 3, SB_SFULL0 = 5, SB_SFREE0 = 7, SB_DRAIN = 9 };
+
+// Two CTAs per SM (98 KB of shared memory and 256 TMEM columns each), so two consumer
+// warpgroups interleave their exp2 work on the MUFU units.
 template <int D, int PASS>
-__global__ void __launch_bounds__(SC_THREADS) score_kernel(SelectArgs a) {
-  __shared__ __align__(16) float kt[SC_KT * D];
-  __shared__ float sbuf[16][SC_KT + 1];
+__global__ void __launch_bounds__(SCT_THREADS, 2) score_tc_kernel(SelectArgs a, uint64_t timeout_ns) {
+  using L = ScoreSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF);
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF + 4);
+  float2* col_mc = (float2*)(smem + L::COL_OFF);  // pass 2: (m, w/Z) per centroid column
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int groups = (a.nQ + 15) / 16;
   const int bh = blockIdx.x / groups;
   const int g = blockIdx.x - bh * groups;
-  const int tid = threadIdx.x;
-  const int ql = tid >> 3, c = tid & 7;
-  const int qb = g * 16 + ql;
-  const bool live = qb < a.nQ;
-  const size_t crow = ((size_t)bh * a.nQ + (live ? qb : 0)) * CMAX + c;
+  const int T = (a.nK + 127) / 128;
 
-  float cr[D];
-  {
-    const uint16_t* cs = a.cent + crow * D;
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[SB_CFULL], 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[SB_FULL0 + b], 128);
+      mbar_init(&bars[SB_EMPTY0 + b], 1);
+      mbar_init(&bars[SB_SFULL0 + b], 1);
+      mbar_init(&bars[SB_SFREE0 + b], 128);
+    }
+    mbar_init(&bars[SB_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------------- producers
+    const int p = tid - 128, u = p & 15, rsub = p >> 4;
+    constexpr int UNITS = D / 8;
+    for (int r = rsub; r < 128; r += 8) {  // centroid rows: 16 query blocks x 8 slots
+      if (u < UNITS) {
+        const int qb = g * 16 + (r >> 3);
+        const bool ok = qb < a.nQ;
+        const uint16_t* src = a.cent + (((size_t)bh * a.nQ + (ok ? qb : 0)) * CMAX + (r & 7)) * D + u * 8;
+        cp_async_16(sbase + L::FIX_OFF + (u >> 3) * L::CHUNK + sw128_off(r, u & 7), src, ok ? 16u : 0u);
+      }
+    }
+    mbar_arrive_cpasync(&bars[SB_CFULL]);
+    const uint16_t* kp = a.Kp + (size_t)bh * a.nK * D;
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1;
+      if (t >= 2 && !mbar_wait(&bars[SB_EMPTY0 + st], ((t >> 1) - 1) & 1, abort_flag, timeout_ns)) break;
+      const uint32_t dst = sbase + L::KP_OFF + st * L::TILE;
+      for (int r = rsub; r < 128; r += 8) {
+        if (u < UNITS) {
+          const int j = t * 128 + r;
+          const bool ok = j < a.nK;
+          cp_async_16(dst + (u >> 3) * L::CHUNK + sw128_off(r, u & 7),
+                      kp + (size_t)(ok ? j : 0) * D + u * 8, ok ? 16u : 0u);
+        }
+      }
+      mbar_arrive_cpasync(&bars[SB_FULL0 + st]);
+    }
+    cp_async_wait_all();
+  } else if (warp == 8) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
+      bool ok = mbar_wait(&bars[SB_CFULL], 0, abort_flag, timeout_ns);
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1;
+        ok = mbar_wait(&bars[SB_FULL0 + st], (t >> 1) & 1, abort_flag, timeout_ns);
+        if (ok && t >= 2) ok = mbar_wait(&bars[SB_SFREE0 + st], ((t >> 1) - 1) & 1, abort_flag, timeout_ns);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t cbase = sbase + L::FIX_OFF;
+        const uint32_t kbase = sbase + L::KP_OFF + st * L::TILE;
 #pragma unroll
-    for (int e = 0; e < D; e += 8) {
-      const uint4 v = live ? __ldg((const uint4*)(cs + e)) : make_uint4(0, 0, 0, 0);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
+          const uint64_t dc = sdesc_sw128(cbase + off, 16, 1024);
+          const uint64_t dk = sdesc_sw128(kbase + off, 16, 1024);
+          if (PASS == 1) umma_f16_ss(tmem + st * 128, dc, dk, IDESC, kk > 0 ? 1u : 0u);
+          else umma_f16_ss(tmem + st * 128, dk, dc, IDESC, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars[SB_SFULL0 + st]);
+        umma_commit(&bars[SB_EMPTY0 + st]);
+      }
+      umma_commit(&bars[SB_DRAIN]);
+      mbar_wait(&bars[SB_DRAIN], 0, abort_flag, timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers (warps 0-3)
+    const int r = tid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (PASS == 2) {  // per-column constants: column r = (query block r>>3, slot r&7)
+      const int qb = g * 16 + (r >> 3);
+      float mm = 0.f, cf = 0.f;
+      if (qb < a.nQ) {
+        const size_t crow = ((size_t)bh * a.nQ + qb) * CMAX + (r & 7);
+        const float Z = a.stats[crow * 2 + 1];
+        mm = a.stats[crow * 2];
+        cf = (Z > 0.f) ? a.w[crow] / Z : 0.f;
+        if (!(mm > -INFINITY)) { mm = 0.f; cf = 0.f; }
+      }
+      col_mc[r] = make_float2(mm, cf);
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 consumer warps only
+    }
+    float m = -INFINITY, z = 0.f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1;
+      ok = mbar_wait(&bars[SB_SFULL0 + st], (t >> 1) & 1, abort_flag, timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sadr = tmem + st * 128 + lane_off;
+      if (PASS == 1) {
+        // online max / sum over 32-column chunks (keeps 32 values live)
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(sadr + c0, v);
+          tmem_wait_ld();
+          float mt = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        cr[e + 2 * k] = bf16_bits_to_float((uint16_t)(w4[k] & 0xffffu));
-        cr[e + 2 * k + 1] = bf16_bits_to_float((uint16_t)(w4[k] >> 16));
+          for (int c = 0; c < 32; ++c) {
+            const float l = (t * 128 + c0 + c < a.nK) ? __uint_as_float(v[c]) * a.scale_log2 : -INFINITY;
+            v[c] = __float_as_uint(l);
+            mt = fmaxf(mt, l);
+          }
+          if (mt > m) {
+            z = (m == -INFINITY) ? 0.f : z * fast_exp2(m - mt);
+            m = mt;
+          }
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc += fast_exp2(__uint_as_float(v[c]) - m);
+          z += acc;
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[SB_SFREE0 + st]);
+      } else {
+        const int j = t * 128 + r;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {  // 4 query blocks per TMEM load
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(sadr + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              // re-read per tile (volatile): hoisting all 128 columns would need 256 registers
+              float mm, cf;
+              asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                           : "=f"(mm), "=f"(cf)
+                           : "r"(smem_u32(col_mc + c0 + q * 8 + c)));
+              acc = fmaf(cf, fast_exp2(fmaf(__uint_as_float(v[q * 8 + c]), a.scale_log2, -mm)), acc);
+            }
+            const int qb = g * 16 + (c0 >> 3) + q;
+            if (j < a.nK && qb < a.nQ) a.S[((size_t)bh * a.nQ + qb) * a.nK + j] = acc;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[SB_SFREE0 + st]);
+      }
+    }
+    if (PASS == 1 && ok) {
+      const int qb = g * 16 + (r >> 3);
+      if (qb < a.nQ) {
+        const size_t crow = ((size_t)bh * a.nQ + qb) * CMAX + (r & 7);
+        a.stats[crow * 2] = m;
+        a.stats[crow * 2 + 1] = z;
       }
     }
   }
-  float m = -INFINITY, z = 0.f, coef = 0.f;
-  if (PASS == 2 && live) {
-    m = a.stats[crow * 2];
-    const float Z = a.stats[crow * 2 + 1];
-    const float wv = a.w[crow];
-    coef = (Z > 0.f) ? wv / Z : 0.f;
-  }
-  const uint16_t* kp = a.Kp + (size_t)bh * a.nK * D;
-  for (int j0 = 0; j0 < a.nK; j0 += SC_KT) {
-    const int nk = min(SC_KT, a.nK - j0);
-    __syncthreads();
-    for (int e = tid; e < SC_KT * D / 2; e += SC_THREADS) {
-      const int kk = e / (D / 2);
-      uint32_t v = 0;
-      if (kk < nk) v = __ldg((const uint32_t*)(kp + (size_t)(j0 + kk) * D) + (e - kk * (D / 2)));
-      kt[2 * e] = bf16_bits_to_float((uint16_t)(v & 0xffffu));
-      kt[2 * e + 1] = bf16_bits_to_float((uint16_t)(v >> 16));
-    }
-    __syncthreads();
-    float l[SC_KT];
-#pragma unroll
-    for (int kk = 0; kk < SC_KT; ++kk) {
-      const float4* kv = (const float4*)(kt + kk * D);
-      float acc = 0.f;
-#pragma unroll
-      for (int e = 0; e < D / 4; ++e) {
-        const float4 x = kv[e];
-        acc = fmaf(cr[4 * e], x.x, acc);
-        acc = fmaf(cr[4 * e + 1], x.y, acc);
-        acc = fmaf(cr[4 * e + 2], x.z, acc);
-        acc = fmaf(cr[4 * e + 3], x.w, acc);
-      }
-      l[kk] = (kk < nk) ? acc * a.scale_log2 : -INFINITY;
-    }
-    if (PASS == 1) {
-      float mt = -INFINITY;
-#pragma unroll
-      for (int kk = 0; kk < SC_KT; ++kk) mt = fmaxf(mt, l[kk]);
-      const float mn = fmaxf(m, mt);
-      float acc = (m == -INFINITY) ? 0.f : z * fast_exp2(m - mn);
-#pragma unroll
-      for (int kk = 0; kk < SC_KT; ++kk) acc += fast_exp2(l[kk] - mn);
-      z = acc;
-      m = mn;
-    } else {
-#pragma unroll
-      for (int kk = 0; kk < SC_KT; ++kk) {
-        float p = coef * fast_exp2(l[kk] - m);
-        p += __shfl_xor_sync(0xffffffffu, p, 4);
-        p += __shfl_xor_sync(0xffffffffu, p, 2);
-        p += __shfl_xor_sync(0xffffffffu, p, 1);
-        if (c == 0) sbuf[ql][kk] = p;
-      }
-      __syncthreads();
-      for (int e = tid; e < 16 * SC_KT; e += SC_THREADS) {
-        const int r = e / SC_KT, kk = e - r * SC_KT;
-        const int q2 = g * 16 + r;
-        if (q2 < a.nQ && kk < nk) a.S[((size_t)bh * a.nQ + q2) * a.nK + j0 + kk] = sbuf[r][kk];
-      }
-    }
-  }
-  if (PASS == 1 && live) {
-    a.stats[crow * 2] = m;
-    a.stats[crow * 2 + 1] = z;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 

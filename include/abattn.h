@@ -131,6 +131,23 @@ ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* 
 ab_status ab_attn_dense(const ab_params* p, const void* Q, const void* K, const void* V,
                         void* O, void* stream);
 
+/* Test and profiling hook (no counterpart on the page): ab_attn with
+ *  - skip_first_arrival != 0: the producers of every CTA never signal their first tile;
+ *    the waiting warps give up after timeout_ns, record AB_ERR_DEVICE_TIMEOUT in the
+ *    status word, drain their copies, free tensor memory and exit (O is undefined);
+ *  - timeout_ns: the limit of every bounded device wait (> 0);
+ *  - trace (device, may be NULL; 8-byte aligned, 3*16*128 uint64, zeroed by the caller):
+ *    a separately compiled traced kernel records clock64() for each pipeline event of
+ *    tiles 0..127 of CTAs 0, 1 and gridDim/3, at trace[(slot*16 + event)*128 + tile];
+ *    events: 0 K copy issued, 1 K arrival, 2 V copy issued, 3 V arrival, 4 K landed (seen
+ *    by the MMA warp), 5 QK issued, 6 V landed, 7 PV issued, 8 softmax tile start,
+ *    9 S ready, 10 P written, 11 CTA end (tile slot 0).
+ * With skip_first_arrival = 0 and trace = NULL it is ab_attn with another wait limit.   */
+ab_status ab_attn_debug(const ab_params* p, const void* Q, const void* K, const void* V,
+                        const int32_t* idx, const float* logpi, int s, void* O,
+                        int skip_first_arrival, uint64_t timeout_ns, uint64_t* trace,
+                        void* stream);
+
 /* Synchronises `stream`, returns the device status word (AB_OK if no device-side problem
  * was recorded since the last call, else the first recorded code) and clears it.       */
 ab_status ab_get_status(void* stream);

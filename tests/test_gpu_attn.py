@@ -125,3 +125,20 @@ def test_bad_index_status():
     keep = [0, 1, 2, 4, 5, 6, 7]
     ref = O.attn_block(np64(Q[0, 0, 128:]), np64(K[0, 0]), np64(V[0, 0]), keep, [0.0] * 7, bk)
     assert_o_close(np64(O_[0, 0, 128:]), ref)
+
+
+def test_device_wait_timeout_is_reported_and_context_survives():
+    """A producer that never signals tile 0: the bounded waits give up after 50 ms, the
+    status word reports AB_ERR_DEVICE_TIMEOUT, and the context stays usable."""
+    H, N, d, bk, s = 1, 256, 64, 4, 64
+    Q, K, V = _qkv(H, N, d, seed=13)
+    idx, lp = random_plan(2, N // bk, s, seed=1)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    O_ = torch.empty(Q.shape, dtype=torch.bfloat16, device="cuda")
+    args = (p, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), lp.cuda(), s, O_)
+    ab.ab_attn_debug(*args, 1, 50_000_000)
+    assert ab.ab_get_status() == -4
+    # the same call without the skipped arrival works afterwards
+    ab.ab_attn_debug(*args, 0, 2_000_000_000)
+    assert ab.ab_get_status() == 0
+    _check(O_.cpu(), Q, K, V, idx, lp, H, N, bk)
