@@ -158,6 +158,17 @@ def kept_flops(w):
     return 4.0 * w.B * w.H * w.N * (w.s * w.kv_block) * w.d
 
 
+def gathered_bytes(w):
+    """K and V bytes one ab_attn call gathers: every query block reads s*bk tokens of each."""
+    return 2.0 * w.B * w.H * w.nQ * (w.s * w.kv_block) * w.d * 2
+
+
+# DRAM bytes per attention launch from the newest ncu capture of the current kernel
+# (dram__bytes_read.sum + dram__bytes_write.sum, scaled from the captured shape to the
+# bench shape by the number of heads); None while the kernel differs from the captured one.
+ATTN_TRAFFIC_BYTES = 3.462e9  # attention v7: 1.0386 GB at 12 heads x 40/12 (profiles/attn_kernel_wan13b.md)
+
+
 def select_plan_bytes(w):
     """Algorithmic HBM bytes of select+plan: |Q| + |K| (bf16) + 2|S| (fp32) + |idx| + |logpi|."""
     qk = 2 * w.B * w.H * w.N * w.d * 2
@@ -291,7 +302,8 @@ def run_ours(args, world, rank, local):
                      "achieved": round(attn_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak_t, 4),
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
-                     "traffic": args.traffic},
+                     "traffic": args.traffic if args.traffic is not None else ATTN_TRAFFIC_BYTES,
+                     "l2_gather_gbs": round(gathered_bytes(w) / (attn_ms * 1e-3) / 1e9, 1)},
         "gpu_launches": args.steps * (4 * run_select + run_plan + reuse * run_attn),
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -25,7 +25,8 @@ def nvcc_cmd(verbose_ptxas: bool = False):
 
 def sources():
     d = os.path.join(HERE, "csrc")
-    return [os.path.join(d, f) for f in os.listdir(d)] + [os.path.join(ROOT, "include", "abattn.h")]
+    return ([os.path.join(d, f) for f in os.listdir(d) if f != "gather_probe.cu"] +
+            [os.path.join(ROOT, "include", "abattn.h")])
 
 
 def up_to_date() -> bool:
@@ -46,6 +47,24 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     return OUT
 
 
+PROBE_SRC = os.path.join(HERE, "csrc", "gather_probe.cu")
+PROBE_OUT = os.path.join(HERE, "gather_probe")
+
+
+def build_probe() -> str:
+    """The L2 gather-bandwidth probe (a stand-alone executable, not part of the library)."""
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", PROBE_SRC,
+           "-o", PROBE_OUT]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError("nvcc failed building gather_probe")
+    return PROBE_OUT
+
+
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
-    print(OUT)
+    if "--probe" in sys.argv:
+        print(build_probe())
+    else:
+        build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
+        print(OUT)

@@ -1,0 +1,132 @@
+// Gather-bandwidth probe: how fast can one B200 SM pull 4-token K/V blocks (4 rows x
+// 256 B = 1 KB, the unit the packed attention gathers) from an L2-resident buffer into
+// shared memory?  This sets the ceiling the attention kernel is measured against.
+//
+//   cpasync : 16-byte cp.async per thread (the attention kernel's copy), 8 warps, one
+//             32 KB tile in flight per CTA
+//   bulk<NT>: 1 KB cp.async.bulk copies completing on an mbarrier, NT tiles in flight
+//
+// Prints cycles per 32 KB tile, bytes/cycle per SM and in aggregate, for grids of 148
+// (one CTA per SM), 74 and 37 CTAs.  Block indices come from a fixed LCG; every address
+// stays inside the 64 MB buffer and every wait is bounded.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <vector>
+
+namespace {
+
+__device__ __forceinline__ uint32_t sa(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__global__ void gather_cpasync(const uint8_t* __restrict__ g, const int* __restrict__ blocks, int nb,
+                               int iters, long long* out) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sbase = sa(sm);
+  const int tid = threadIdx.x;
+  const long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    for (int c = tid; c < 2048; c += blockDim.x) {
+      const int r = c >> 4, u = c & 15;
+      const int blk = blocks[((blockIdx.x * iters + it) * 32 + (r >> 2)) % nb];
+      const uint8_t* src = g + ((size_t)blk * 4 + (r & 3)) * 256 + u * 16;
+      const uint32_t dst = sbase + (u >> 3) * 16384 + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+  }
+  if (tid == 0) out[blockIdx.x] = clock64() - t0;
+}
+
+template <int NT>
+__global__ void gather_bulk(const uint8_t* __restrict__ g, const int* __restrict__ blocks, int nb,
+                            int iters, long long* out, int* err) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  __shared__ __align__(8) uint64_t bar[NT];
+  const int tid = threadIdx.x;  // one warp: lane l copies block l of each tile
+  if (tid == 0) {
+    for (int i = 0; i < NT; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sa(&bar[i])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int it) {
+    const int st = it % NT;
+    if (tid == 0)
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sa(&bar[st])), "r"(32768)
+                   : "memory");
+    __syncwarp();
+    const int blk = blocks[((blockIdx.x * iters + it) * 32 + tid) % nb];
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::"r"(
+            sa(sm) + st * 32768 + tid * 1024),
+        "l"(g + (size_t)blk * 1024), "r"(sa(&bar[st]))
+        : "memory");
+  };
+  const long long t0 = clock64();
+  for (int it = 0; it < NT && it < iters; ++it) issue(it);
+  for (int it = 0; it < iters; ++it) {
+    const int st = it % NT;
+    uint32_t ok = 0;
+    for (long long k = 0; k < 20000000 && !ok; ++k)
+      asm volatile(
+          "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0,1,0,p; }"
+          : "=r"(ok)
+          : "r"(sa(&bar[st])), "r"((it / NT) & 1)
+          : "memory");
+    if (!ok && tid == 0) atomicExch(err, 1);
+    __syncwarp();
+    if (it + NT < iters) issue(it + NT);
+  }
+  if (tid == 0) out[blockIdx.x] = clock64() - t0;
+}
+
+}  // namespace
+
+int main() {
+  const size_t G = 64ull << 20;
+  const int nblocks = (int)(G / 1024);
+  uint8_t* g = nullptr;
+  int* blocks = nullptr;
+  long long* out = nullptr;
+  int* err = nullptr;
+  if (cudaMalloc(&g, G) != cudaSuccess) return 1;
+  cudaMemset(g, 1, G);
+  std::vector<int> hb(1 << 20);
+  uint32_t x = 12345;
+  for (auto& b : hb) {
+    x = x * 1664525u + 1013904223u;
+    b = (int)(x % (uint32_t)nblocks);
+  }
+  cudaMalloc(&blocks, hb.size() * 4);
+  cudaMemcpy(blocks, hb.data(), hb.size() * 4, cudaMemcpyHostToDevice);
+  cudaMalloc(&out, 148 * 8);
+  cudaMalloc(&err, 4);
+  cudaMemset(err, 0, 4);
+  const int iters = 64;  // (147*64 + 63)*32 + 31 < 2^20 entries
+  auto report = [&](const char* name, int grid) {
+    cudaDeviceSynchronize();
+    std::vector<long long> h(grid);
+    cudaMemcpy(h.data(), out, grid * 8, cudaMemcpyDeviceToHost);
+    double avg = 0;
+    for (auto v : h) avg += (double)v;
+    avg /= grid;
+    printf("grid %3d %-10s %7.0f cycles/32KB tile  %5.1f B/cycle/SM  aggregate %6.0f B/cycle\n", grid, name,
+           avg / iters, 32768.0 * iters / avg, grid * 32768.0 * iters / avg);
+  };
+  cudaFuncSetAttribute(gather_cpasync, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * 1024);
+  cudaFuncSetAttribute(gather_bulk<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024);
+  cudaFuncSetAttribute(gather_bulk<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+  for (int grid : {148, 74, 37}) {
+    for (int rep = 0; rep < 2; ++rep) gather_cpasync<<<grid, 256, 33 * 1024>>>(g, blocks, (int)hb.size(), iters, out);
+    report("cpasync", grid);
+    for (int rep = 0; rep < 2; ++rep) gather_bulk<1><<<grid, 32, 32 * 1024>>>(g, blocks, (int)hb.size(), iters, out, err);
+    report("bulk x1", grid);
+    for (int rep = 0; rep < 2; ++rep) gather_bulk<4><<<grid, 32, 128 * 1024>>>(g, blocks, (int)hb.size(), iters, out, err);
+    report("bulk x4", grid);
+  }
+  int herr = 0;
+  cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);
+  printf("bulk wait timeouts: %d; status: %s\n", herr, cudaGetErrorString(cudaGetLastError()));
+  return herr != 0;
+}
