@@ -30,6 +30,8 @@
 // drains and exits.
 #pragma once
 
+#include <climits>
+
 #include "common.cuh"
 
 namespace abattn {
@@ -57,7 +59,8 @@ struct AttnArgs {
 // Event tracing (TRACE builds only): CTAs 0, 1 and the one at a third of the grid record
 // clock64() per tile for the events below into trace[((slot * 16) + event) * 128 + t].
 enum { EV_COPY_START = 0, EV_COPY_ISSUED, EV_SM_LOADED, EV_SM_MAX, EV_LANDED, EV_QK,
-       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_COUNT };
+       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_SM_SFULL,
+       EV_SM_PDONE_W1, EV_SM_PDONE_W2, EV_SM_PDONE_W3, EV_COUNT };
 constexpr int TRACE_TILES = 128;
 
 template <int D>
@@ -149,23 +152,33 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     const int nb = 128 >> a.bk_shift;  // sampled blocks per tile
 
     // Block indices of one tile, spread over the warp: lane e (+32k) holds the tile's
-    // block e (-1 for padding or a rejected entry).  Loaded coalesced one tile ahead and
-    // broadcast to the copying lanes with shuffles.
+    // block e.  Loaded raw and coalesced one tile ahead (nothing branches on a loaded value
+    // until the next tile, so the loads stay in flight), checked once per tile, and
+    // broadcast to the copying lanes with shuffles; -1 marks padding or a rejected entry.
+    constexpr int PAD = INT_MIN;
     int jc[4], jn[4];
     auto fetch = [&](int t, int (&jr)[4]) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int e = lane + 32 * k;
         const int m = t * nb + e;
-        jr[k] = -1;
-        if (!DENSE && e < nb && m < a.s) {
-          const int j = __ldg(a.idx + plan_off + m);
-          if (j < 0 || j >= a.nK) ab_flag(AB_ERR_DEVICE_CHECK);
-          else jr[k] = j;
-        }
+        jr[k] = (!DENSE && e < nb && m < a.s) ? __ldg(a.idx + plan_off + m) : PAD;
       }
     };
-    if (!DENSE) fetch(0, jc);
+    auto check = [&](int (&jr)[4]) {
+      bool bad = false;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const bool ok = jr[k] >= 0 && jr[k] < a.nK;
+        bad |= (jr[k] != PAD) && !ok;
+        jr[k] = ok ? jr[k] : -1;
+      }
+      if (bad) ab_flag(AB_ERR_DEVICE_CHECK);
+    };
+    if (!DENSE) {
+      fetch(0, jc);
+      check(jc);
+    }
 
     // Q tile: rows row0..row0+127 (zero beyond N)
     for (int r = rsub; r < 128; r += 8) {
@@ -230,9 +243,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         if (a.debug_skip_arrive && t == 0) continue;  // test knob: never signal tile 0
         mbar_arrive_cpasync(&bars[(half ? B_VFULL0 : B_KFULL0) + st]);
       }
-      if (!DENSE) {
+      if (!DENSE && t + 1 < T) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) jc[k] = jn[k];
+        check(jc);
       }
       st = (st + 1 == ATTN_STAGES) ? 0 : st + 1;
       if (p == 0) ev(EV_COPY_ISSUED, t);
@@ -315,18 +329,16 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     bool ok = true;
     const size_t plan_off = (size_t)blockIdx.x * a.s;
     const int nb = 128 >> a.bk_shift;
-    // column r's plan entry for tile t: its block index (or -1) and log pi
+    // column r's plan entry for tile t as loaded (block index, log pi), -1 past the end of
+    // the sample; both loads are unconditional so they stay in flight until the next tile
     auto entry = [&](int t, int& j, float& lp) {
       j = -1;
       lp = 0.f;
       if (!DENSE) {
         const int m = t * nb + (r >> a.bk_shift);
         if (m < a.s) {
-          const int jj = __ldg(a.idx + plan_off + m);
-          if (jj >= 0 && jj < a.nK) {
-            j = jj;
-            lp = __ldg(a.logpi + plan_off + m);
-          }
+          j = __ldg(a.idx + plan_off + m);
+          lp = __ldg(a.logpi + plan_off + m);
         }
       }
     };
@@ -341,15 +353,16 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         if (DENSE) {
           b2 = (t * 128 + r < a.N) ? 0.f : -INFINITY;
         } else {
-          const bool valid = jcol >= 0 && jcol * a.bk + (r & (a.bk - 1)) < a.N;
+          const bool valid = jcol >= 0 && jcol < a.nK && jcol * a.bk + (r & (a.bk - 1)) < a.N;
           b2 = valid ? -lcol * LOG2E : -INFINITY;
         }
         bias[st * 128 + r] = b2;
         mbar_arrive(&bars[B_BIAS0 + st]);
         if (t + 1 < T) entry(t + 1, jnext, lnext);
       }
-      ok = mbar_wait(&bars[B_SFULL0 + st], (t >> 1) & 1, abort_flag, a.timeout_ns) &&
-           mbar_wait(&bars[B_BIAS0 + st], (t >> 1) & 1, abort_flag, a.timeout_ns);
+      ok = mbar_wait(&bars[B_SFULL0 + st], (t >> 1) & 1, abort_flag, a.timeout_ns);
+      if (r == 0) ev(EV_SM_SFULL, t);
+      ok = ok && mbar_wait(&bars[B_BIAS0 + st], (t >> 1) & 1, abort_flag, a.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       if (r == 0) ev(EV_SM_READY, t);
@@ -438,7 +451,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_PFULL0 + st]);
-      if (r == 0) ev(EV_SM_PDONE, t);
+      if (lane == 0) ev(warp == 0 ? EV_SM_PDONE : EV_SM_PDONE_W1 + warp - 1, t);
       jcol = jnext;
       lcol = lnext;
     }

@@ -106,11 +106,15 @@ AB_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity.  Gives up when *abort is raised
 // by another thread of the CTA, or after timeout_ns (then records
 // AB_ERR_DEVICE_TIMEOUT and raises *abort).  Returns true when the phase completed.
+// Spins on the non-suspending probe: a thread parked in try_wait was observed to resume
+// only long after an arrival made by tcgen05.commit.
 AB_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int k = 0; k < 64; ++k)
+      if (mbar_test(bar, parity)) return true;
     if (*abort) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
       ab_flag(AB_ERR_DEVICE_TIMEOUT);

@@ -56,12 +56,23 @@ AB_DEV uint32_t philox4x32_10_w0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t
   return c0;
 }
 
+// floor(x * 2^32) for 0 <= x < 1, exactly, from the fp32 bit pattern: x = m 2^(e-150) with
+// the 24-bit significand m, so x 2^32 = m 2^(e-118) (at most 2^32 - 2^8: fits 32 bits).
+AB_DEV uint32_t frac32(float x) {
+  const uint32_t b = __float_as_uint(x);
+  const int e = (int)(b >> 23);
+  const uint32_t m = (b & 0x7FFFFFu) | 0x800000u;
+  if (e >= 118) return m << (e - 118);
+  const int sh = 118 - e;
+  return sh < 32 ? (m >> sh) : 0u;  // also 0 for zero and subnormal x (far below 2^-32)
+}
+
 // q_j(lambda) in 2^-32 units.  __fmul_rn keeps the product a single fp32 rounding.
 AB_DEV uint64_t fixed_q(float lam, float sv) {
   if (!(sv > 0.f)) return 0ull;
   const float x = __fmul_rn(lam, sv);
   if (x >= 1.0f) return TWO32;
-  return (uint64_t)__float2ull_rz(__fmul_rn(x, 4294967296.0f));  // exact scaling, truncation
+  return (uint64_t)frac32(x);
 }
 
 // Block-wide sum of a uint64 (all threads get the result).  red: PLAN_WARPS slots.
@@ -78,18 +89,21 @@ AB_DEV uint64_t block_sum_u64(uint64_t v, uint64_t* red) {
   return tot;
 }
 
-// Block-wide fp32 sum (all threads get the result).
-AB_DEV float block_sum_f32(float v, float* red) {
+// Block-wide sums of a (uint64 count, fp64 value) pair, one pair of barriers.
+AB_DEV void block_sum_cd(uint64_t& c, double& v, uint64_t* redc, double* redv) {
 #pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  for (int o = 16; o; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    v += __shfl_xor_sync(0xffffffffu, v, o);
+  }
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   __syncthreads();
-  if (l == 0) red[w] = v;
+  if (l == 0) { redc[w] = c; redv[w] = v; }
   __syncthreads();
-  float tot = 0.f;
+  c = 0;
+  v = 0.0;
 #pragma unroll
-  for (int i = 0; i < PLAN_WARPS; ++i) tot += red[i];
-  return tot;
+  for (int i = 0; i < PLAN_WARPS; ++i) { c += redc[i]; v += redv[i]; }
 }
 
 // Exclusive block scan of uint64 values in thread order; returns this thread's prefix.
@@ -119,14 +133,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   extern __shared__ float srow_smem[];
   __shared__ uint64_t red[PLAN_WARPS];
   __shared__ uint64_t red2[PLAN_WARPS];
-  __shared__ float redf[PLAN_WARPS];
+  __shared__ double redd[PLAN_WARPS];
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nK = a.nK;
   const float* grow = a.S + (size_t)row * nK;
   const float* srow = grow;
+  const int nK4 = (nK + 3) >> 2;  // staged row padded with zeros to whole float4s
   if (STAGED) {
-    for (int j = tid; j < nK; j += PLAN_THREADS) srow_smem[j] = __ldg(grow + j);
+    for (int j = tid; j < nK4 * 4; j += PLAN_THREADS) srow_smem[j] = (j < nK) ? __ldg(grow + j) : 0.f;
     __syncthreads();
     srow = srow_smem;
   }
@@ -141,55 +156,108 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   auto F = [&](uint32_t bits) -> uint64_t {
     const float lam = __uint_as_float(bits);
     uint64_t part = 0;
-    for (int j = tid; j < nK; j += PLAN_THREADS) part += fixed_q(lam, srow[j]);
+    if (STAGED) {
+      const float4* s4 = reinterpret_cast<const float4*>(srow);
+      for (int j = tid; j < nK4; j += PLAN_THREADS) {
+        const float4 v = s4[j];
+        part += fixed_q(lam, v.x) + fixed_q(lam, v.y) + fixed_q(lam, v.z) + fixed_q(lam, v.w);
+      }
+    } else {
+      for (int j = tid; j < nK; j += PLAN_THREADS) part += fixed_q(lam, srow[j]);
+    }
     return block_sum_u64(part, red);
   };
   uint32_t lo = 0u, hi = 0x7F800000u;
-  const bool reachable = F(hi) >= target;
+  // positive blocks and their total score; fewer than s positive blocks = budget unreachable
+  // per-thread sums in compensated fp32 (no per-element fp64 conversions), block sum in fp64
+  uint64_t npos = 0;
+  double tot = 0.0;
+  {
+    float sum = 0.f, comp = 0.f;
+    for (int j = tid; j < nK; j += PLAN_THREADS) {
+      const float sv = srow[j];
+      if (sv > 0.f) {
+        const float y = sv - comp, t2 = sum + y;
+        comp = (t2 - sum) - y;
+        sum = t2;
+        ++npos;
+      }
+    }
+    tot = (double)sum - (double)comp;
+  }
+  block_sum_cd(npos, tot, red, redd);
+  const bool reachable = npos >= s;
   if (reachable) {
-    // water-filling estimate in fp32 (only a starting point)
-    float lam_est = 0.f;
-    {
-      float part = 0.f;
-      for (int j = tid; j < nK; j += PLAN_THREADS) part += fmaxf(srow[j], 0.f);
-      float tot = block_sum_f32(part, redf);
-      lam_est = (tot > 0.f) ? (float)a.s / tot : 0.f;
-      for (int it = 0; it < 8 && lam_est > 0.f && isfinite(lam_est); ++it) {
-        float rest = 0.f;
-        uint32_t nsat = 0;
+    // Water filling in fp64 (a starting point only): lambda <- (s - |saturated|) / (sum of
+    // the unsaturated scores) until the saturated set stops growing; in practice a few
+    // rounds, ending within an ulp or two of lambda*.
+    double lam_w = (tot > 0.0) ? (double)a.s / tot : 0.0;
+    double rest_est = tot;
+    for (int it = 0; it < 32 && lam_w > 0.0; ++it) {
+      uint64_t nsat = 0;
+      double rest = 0.0;
+      const float lw = (float)lam_w;
+      {
+        float sum = 0.f, comp = 0.f;
         for (int j = tid; j < nK; j += PLAN_THREADS) {
           const float sv = srow[j];
           if (sv > 0.f) {
-            if (__fmul_rn(lam_est, sv) >= 1.f) ++nsat; else rest += sv;
+            if (__fmul_rn(lw, sv) >= 1.f) {
+              ++nsat;
+            } else {
+              const float y = sv - comp, t2 = sum + y;
+              comp = (t2 - sum) - y;
+              sum = t2;
+            }
           }
         }
-        const uint64_t ns = block_sum_u64(nsat, red);
-        rest = block_sum_f32(rest, redf);
-        if (ns >= (uint64_t)a.s || !(rest > 0.f)) break;
-        const float nxt = (float)((uint64_t)a.s - ns) / rest;
-        if (!(nxt > lam_est)) break;  // converged (the iteration only increases)
-        lam_est = nxt;
+        rest = (double)sum - (double)comp;
       }
+      block_sum_cd(nsat, rest, red, redd);
+      rest_est = rest;
+      if (nsat >= (uint64_t)a.s || !(rest > 0.0)) break;
+      const double nxt = (double)((uint64_t)a.s - nsat) / rest;
+      if (!(nxt > lam_w)) break;  // converged (the iteration only increases)
+      lam_w = nxt;
     }
+    const float lam_est = (float)lam_w;
     uint32_t b = __float_as_uint(lam_est);
     if (!(lam_est > 0.f) || !isfinite(lam_est)) b = 0x3F800000u;  // 1.0: any start works
-    if (F(b) >= target) {  // boundary at or below b: step down
-      hi = b;
-      uint32_t step = 1;
-      while (true) {
-        const uint32_t cand = (hi > step) ? hi - step : 0u;
-        if (cand == 0u || F(cand) < target) { lo = cand; break; }
-        hi = cand;
-        step <<= 1;
+    uint64_t fb = F(b);
+    // one Newton step on the fixed-point sum: F grows by about rest * 2^32 per unit lambda
+    if (rest_est > 0.0 && isfinite(lam_est) && lam_est > 0.f) {
+      const double lam_n = (double)__uint_as_float(b) +
+                           ((double)target - (double)fb) / (rest_est * 4294967296.0);
+      const float lf = (float)lam_n;
+      if (lf > 0.f && isfinite(lf) && __float_as_uint(lf) != b) {
+        const uint32_t b2 = __float_as_uint(lf);
+        const uint64_t f2 = F(b2);
+        // keep whichever point is on the same side as the boundary search needs
+        if ((f2 >= target) == (fb >= target)) { b = b2; fb = f2; }
+        else if (b2 > b) { lo = b; hi = b2; }
+        else { lo = b2; hi = b; }
       }
-    } else {  // boundary above b: step up
-      lo = b;
-      uint32_t step = 1;
-      while (true) {
-        const uint32_t cand = (0x7F800000u - lo > step) ? lo + step : 0x7F800000u;
-        if (cand == 0x7F800000u || F(cand) >= target) { hi = cand; break; }
-        lo = cand;
-        step <<= 1;
+    }
+    const bool bracketed = !(lo == 0u && hi == 0x7F800000u);  // by the Newton point
+    if (!bracketed) {
+      if (fb >= target) {  // boundary at or below b: step down
+        hi = b;
+        uint32_t step = 1;
+        while (true) {
+          const uint32_t cand = (hi > step) ? hi - step : 0u;
+          if (cand == 0u || F(cand) < target) { lo = cand; break; }
+          hi = cand;
+          step <<= 1;
+        }
+      } else {  // boundary above b: step up
+        lo = b;
+        uint32_t step = 1;
+        while (true) {
+          const uint32_t cand = (0x7F800000u - lo > step) ? lo + step : 0x7F800000u;
+          if (cand == 0x7F800000u || F(cand) >= target) { hi = cand; break; }
+          lo = cand;
+          step <<= 1;
+        }
       }
     }
     while (hi - lo > 1u) {
@@ -286,10 +354,22 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       if (sel) {
         if (o < s) {
           oidx[o] = j;
-          olp[o] = (qq == TWO32) ? 0.f : (float)log((double)qq * (1.0 / 4294967296.0));
+          // the probability's fixed-point value for now (2^32 - 1 stands for pi = 1: a capped
+          // or ordinary q is at most 2^32 - 256); its log follows in a compacted pass
+          reinterpret_cast<uint32_t*>(olp)[o] = (qq == TWO32) ? 0xFFFFFFFFu : (uint32_t)qq;
         }
         ++o;
       }
+    }
+  }
+  // log(pi) for the s outputs, spread evenly over the threads (no divergent fp64 log)
+  __syncthreads();
+  {
+    float* olp = a.logpi + (size_t)row * a.s;
+    uint32_t* raw = reinterpret_cast<uint32_t*>(olp);
+    for (int o = tid; o < a.s; o += PLAN_THREADS) {
+      const uint32_t q = raw[o];
+      olp[o] = (q == 0xFFFFFFFFu) ? 0.f : (float)log((double)q * (1.0 / 4294967296.0));
     }
   }
 }

@@ -75,14 +75,30 @@ __global__ void pool_kernel(SelectArgs a) {
 }
 
 // ------------------------------------------------------------------ k-means
+//
+// One CTA of 256 threads per (bh, query block).
+//  * Segment means (the start) and member means (the update) are exact fp64 sums of the
+//    bf16 rows divided by the count (IEEE division), as the CPU reference computes them.
+//    The update visits the rows in label order (a counting sort), so each thread (one
+//    dimension) runs through the rows once, accumulating into the current cluster.
+//  * Assignment: two threads per row compute the 8 squared distances in fp32 against the
+//    fp32-rounded centroids.  With u = 2^-24 and n = d terms, the fp32 distance differs
+//    from the exact one by at most (n + 4) u (2 |q|^2 + 2 |c|^2) (rounding of c, of q - c,
+//    and of the n-term sum), so when the best and second-best fp32 distances are further
+//    apart than the sum of their bounds the fp32 choice is the exact argmin.  Rows inside
+//    the margin are recomputed in fp64 (ties to the lowest cluster), like the reference.
 
 template <int D>
 __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   __shared__ __align__(16) uint16_t qs[128 * D];
   __shared__ double c64[CMAX * D];
+  __shared__ __align__(16) float cf[CMAX * D];
+  __shared__ float c2[CMAX];
   __shared__ int cnt[CMAX];
+  __shared__ int off[CMAX];
   __shared__ int alive[CMAX];
   __shared__ int8_t lab[128];
+  __shared__ uint8_t perm[128];
   const int bq = blockIdx.x;  // bh * nQ + i
   const int bh = bq / a.nQ, i = bq - bh * a.nQ;
   const int row0 = i * 128;
@@ -90,10 +106,10 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   const int tid = threadIdx.x;
   const int C = a.C;
   constexpr int UNITS = D / 8;
+  constexpr int H = D / 2;  // dimensions per thread in the assignment
 
   const uint16_t* qsrc = a.Q + ((size_t)bh * a.N + row0) * D;
-  for (int e = tid; e < n * UNITS; e += KM_THREADS)
-    ((uint4*)qs)[e] = __ldg((const uint4*)qsrc + e);
+  for (int e = tid; e < n * UNITS; e += KM_THREADS) ((uint4*)qs)[e] = __ldg((const uint4*)qsrc + e);
   if (tid < CMAX) {
     const int s0 = tid * n / C, s1 = (tid + 1) * n / C;
     cnt[tid] = (tid < C) ? s1 - s0 : 0;
@@ -107,7 +123,7 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
     lab[tid] = (int8_t)c;
   }
   __syncthreads();
-  // segment means (fp64)
+  // segment means (fp64, exact sums)
   for (int p = tid; p < CMAX * D; p += KM_THREADS) {
     const int c = p / D, dd = p - c * D;
     double acc = 0.0;
@@ -120,47 +136,123 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   }
   __syncthreads();
 
+  const int ar = tid >> 1;   // assignment: row
+  const int ah = tid & 1;    // ... and which half of the dimensions
   for (int it = 0; it < a.iters; ++it) {
-    // assignment: thread r owns query row r (kept in registers)
-    if (tid < n) {
-      uint32_t qr[D / 2];
+    // fp32 copies of the centroids and their squared norms
+    for (int p = tid; p < CMAX * D; p += KM_THREADS) cf[p] = (float)c64[p];
+    __syncthreads();
+    if (tid < 32) {
 #pragma unroll
-      for (int e = 0; e < D / 8; ++e) {
-        const uint4 v = ((const uint4*)(qs + tid * D))[e];
-        qr[4 * e] = v.x; qr[4 * e + 1] = v.y; qr[4 * e + 2] = v.z; qr[4 * e + 3] = v.w;
+      for (int c = 0; c < CMAX; ++c) {
+        float part = 0.f;
+        for (int dd = tid; dd < D; dd += 32) part = fmaf(cf[c * D + dd], cf[c * D + dd], part);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (tid == 0) c2[c] = part;
       }
-      double best = 0.0;
-      int bc = -1;
-      for (int c = 0; c < C; ++c) {
-        if (!alive[c]) continue;
-        const double* cc = c64 + c * D;
-        double dist = 0.0;
+    }
+    __syncthreads();
+    // assignment (rows >= n take part in the shuffles but are not stored)
+    {
+      const uint16_t* qrow = qs + (ar < n ? ar : 0) * D + ah * H;
+      float dist[CMAX];
 #pragma unroll
-        for (int e = 0; e < D / 2; ++e) {
-          const double d0 = bf16_to_double((uint16_t)(qr[e] & 0xffffu)) - cc[2 * e];
-          const double d1 = bf16_to_double((uint16_t)(qr[e] >> 16)) - cc[2 * e + 1];
-          dist = fma(d0, d0, dist);
-          dist = fma(d1, d1, dist);
+      for (int c = 0; c < CMAX; ++c) dist[c] = 0.f;
+      float q2 = 0.f;
+#pragma unroll 4
+      for (int e = 0; e < H; e += 8) {
+        const uint4 v = *(const uint4*)(qrow + e);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        float qv[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          qv[2 * k] = __uint_as_float(w4[k] << 16);
+          qv[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
         }
-        if (bc < 0 || dist < best) { best = dist; bc = c; }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) q2 = fmaf(qv[k], qv[k], q2);
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) {
+          const float* cc = cf + c * D + ah * H + e;
+          const float4 c0 = *(const float4*)cc;
+          const float4 c1 = *(const float4*)(cc + 4);
+          const float dv[8] = {qv[0] - c0.x, qv[1] - c0.y, qv[2] - c0.z, qv[3] - c0.w,
+                               qv[4] - c1.x, qv[5] - c1.y, qv[6] - c1.z, qv[7] - c1.w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) dist[c] = fmaf(dv[k], dv[k], dist[c]);
+        }
       }
-      lab[tid] = (int8_t)bc;
+#pragma unroll
+      for (int c = 0; c < CMAX; ++c) dist[c] += __shfl_xor_sync(0xffffffffu, dist[c], 1);
+      q2 += __shfl_xor_sync(0xffffffffu, q2, 1);
+      int best = -1, second = -1;
+      float d1 = 0.f, d2 = 0.f, n1 = 0.f, n2 = 0.f;  // best / second distance and |c|^2
+#pragma unroll
+      for (int c = 0; c < CMAX; ++c) {
+        if (!alive[c]) continue;
+        if (best < 0 || dist[c] < d1) {
+          second = best; d2 = d1; n2 = n1;
+          best = c; d1 = dist[c]; n1 = c2[c];
+        } else if (second < 0 || dist[c] < d2) {
+          second = c; d2 = dist[c]; n2 = c2[c];
+        }
+      }
+      constexpr float U = 5.9604645e-8f;  // 2^-24
+      bool certain = true;
+      if (second >= 0) {
+        const float kb = (float)(D + 4) * U * 2.f * 1.0625f;  // bound factor with margin
+        certain = d2 - d1 > kb * ((q2 + n1) + (q2 + n2));
+      }
+      // rows whose fp32 margin is too small: recompute all distances in fp64
+      if (__any_sync(0xffffffffu, !certain && ar < n)) {
+        double dd64[CMAX];
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) dd64[c] = 0.0;
+        if (!certain) {
+          for (int e = 0; e < H; ++e) {
+            const double qd = bf16_to_double(qrow[e]);
+#pragma unroll
+            for (int c = 0; c < CMAX; ++c) {
+              const double dv = qd - c64[c * D + ah * H + e];
+              dd64[c] = fma(dv, dv, dd64[c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) dd64[c] += __shfl_xor_sync(0xffffffffu, dd64[c], 1);
+        if (!certain) {
+          best = -1;
+          double b64 = 0.0;
+#pragma unroll
+          for (int c = 0; c < CMAX; ++c)
+            if (alive[c] && (best < 0 || dd64[c] < b64)) { best = c; b64 = dd64[c]; }
+        }
+      }
+      if (ah == 0 && ar < n) lab[ar] = (int8_t)best;
+    }
+    if (tid < CMAX) cnt[tid] = 0;
+    __syncthreads();
+    if (tid < n) atomicAdd(&cnt[lab[tid]], 1);
+    __syncthreads();
+    if (tid == 0) {
+      int o = 0;
+      for (int c = 0; c < CMAX; ++c) { off[c] = o; o += cnt[c]; }
     }
     __syncthreads();
-    if (tid < CMAX) {
-      int k = 0;
-      for (int r = 0; r < n; ++r) k += (lab[r] == tid);
-      cnt[tid] = k;
-    }
+    if (tid < n) perm[atomicAdd(&off[lab[tid]], 1)] = (uint8_t)tid;  // off[c] ends at its cluster's end
     __syncthreads();
-    // update: fp64 member means; empty clusters keep their previous centroid
-    for (int p = tid; p < CMAX * D; p += KM_THREADS) {
-      const int c = p / D, dd = p - c * D;
-      if (cnt[c] > 0) {
-        double acc = 0.0;
-        for (int r = 0; r < n; ++r)
-          if (lab[r] == c) acc += bf16_to_double(qs[r * D + dd]);
-        c64[p] = acc / (double)cnt[c];
+    // update: each thread owns a dimension and walks the rows grouped by cluster
+    if (tid < D) {
+      int r0 = 0;
+      for (int c = 0; c < CMAX; ++c) {
+        const int k = cnt[c];
+        if (k > 0) {
+          double acc = 0.0;
+          for (int q = r0; q < r0 + k; ++q) acc += bf16_to_double(qs[perm[q] * D + tid]);
+          c64[c * D + tid] = acc / (double)k;
+        }
+        r0 += k;
       }
     }
     __syncthreads();
@@ -177,7 +269,6 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   if (tid < CMAX) a.w[(size_t)bq * CMAX + tid] = alive[tid] ? (float)((double)cnt[tid] / (double)n) : 0.f;
   if (a.labels && tid < 128) a.labels[(size_t)bh * a.nQ * 128 + row0 + tid] = (tid < n) ? lab[tid] : (int8_t)-1;
 }
-
 
 // ------------------------------------------------------------------ block scores (tcgen05)
 //
