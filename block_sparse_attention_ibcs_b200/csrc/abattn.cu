@@ -165,6 +165,7 @@ ab_status run_attn(const Dims& d, const void* Q, const void* K, const void* V, c
   a.bk_shift = ilog2_exact(d.bk);
   a.ntiles = DENSE ? (int)((d.N + 127) / 128) : (int)(((long long)s * d.bk + 127) / 128);
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  a.sqrt_d = (float)sqrt((double)D);
   a.timeout_ns = timeout_ns;
   a.debug_skip_arrive = debug_skip;
   a.trace = trace;

@@ -243,6 +243,19 @@ AB_DEV uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_byt
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle (layout type 0).  K-major canonical
+// layout of 8-row x 16-byte core matrices, each stored as 128 contiguous bytes (row i at
+// byte 16 i):  sbo = byte distance between core matrices adjacent in M/N (the next 8
+// rows), lbo = byte distance between core matrices adjacent in K (the next 8 elements).
+AB_DEV uint64_t sdesc_noswizzle(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 D, dense.
 //   a_mn / b_mn: 0 = K-major, 1 = MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
