@@ -16,7 +16,14 @@
 //   offset_hi, 0)).
 //
 // One CTA of PLAN_THREADS threads per row.  The row is staged in shared memory when it
-// fits, otherwise re-read from global memory (L2) on each bisection step.
+// fits, otherwise re-read from global memory (L2) on each pass.  Passes over the row:
+// staging with the positive count and sum; a water-filling estimate of lambda (usually
+// one pass); F at the estimate and at one Newton step from it (these bracket lambda* to
+// one ulp on typical rows; otherwise a doubling search and bisection follow); the codes
+// (q_j or "saturated") with per-thread sums; and the output pass.  The number selected
+// in each thread's contiguous chunk needs no pass of its own: non-saturated intervals are
+// shorter than 2^32, so the chunk's blocks hold exactly the lattice points of the chunk's
+// (contiguous) interval.
 #pragma once
 
 #include "common.cuh"
@@ -56,23 +63,24 @@ AB_DEV uint32_t philox4x32_10_w0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t
   return c0;
 }
 
-// floor(x * 2^32) for 0 <= x < 1, exactly, from the fp32 bit pattern: x = m 2^(e-150) with
-// the 24-bit significand m, so x 2^32 = m 2^(e-118) (at most 2^32 - 2^8: fits 32 bits).
-AB_DEV uint32_t frac32(float x) {
+// q_j(lambda) = floor(fl32(lambda * S_j) * 2^32) for fl32(lambda S_j) < 1, exactly, from
+// the fp32 bit pattern: x = m 2^(e-150) with the 24-bit significand m, so x 2^32 =
+// (m 2^8) >> (126 - e); (b << 8) | 2^31 is m 2^8, and the clamping funnel shift turns
+// shifts of 32 or more into 0 (x < 2^-32 or zero; a negative or NaN x wraps to such a
+// shift too, so scores that are not positive contribute 0).  Returns whether x >= 1, where
+// q_j = 2^32 instead.  __fmul_rn keeps the product a single fp32 rounding.
+AB_DEV bool fixed_q32(float lam, float sv, uint32_t& q) {
+  const float x = __fmul_rn(lam, sv);
   const uint32_t b = __float_as_uint(x);
-  const int e = (int)(b >> 23);
-  const uint32_t m = (b & 0x7FFFFFu) | 0x800000u;
-  if (e >= 118) return m << (e - 118);
-  const int sh = 118 - e;
-  return sh < 32 ? (m >> sh) : 0u;  // also 0 for zero and subnormal x (far below 2^-32)
+  q = __funnelshift_rc((b << 8) | 0x80000000u, 0u, 126u - (b >> 23));
+  return x >= 1.0f;
 }
 
-// q_j(lambda) in 2^-32 units.  __fmul_rn keeps the product a single fp32 rounding.
-AB_DEV uint64_t fixed_q(float lam, float sv) {
-  if (!(sv > 0.f)) return 0ull;
-  const float x = __fmul_rn(lam, sv);
-  if (x >= 1.0f) return TWO32;
-  return (uint64_t)frac32(x);
+// F's per-thread part: saturated blocks add 2^32, the others q_j.
+AB_DEV void add_q(float lam, float sv, uint64_t& acc) {
+  uint32_t q;
+  const bool sat = fixed_q32(lam, sv, q);
+  acc += sat ? TWO32 : (uint64_t)q;
 }
 
 // Block-wide sum of a uint64 (all threads get the result).  red: PLAN_WARPS slots.
@@ -106,26 +114,42 @@ AB_DEV void block_sum_cd(uint64_t& c, double& v, uint64_t* redc, double* redv) {
   for (int i = 0; i < PLAN_WARPS; ++i) { c += redc[i]; v += redv[i]; }
 }
 
-// Exclusive block scan of uint64 values in thread order; returns this thread's prefix.
-AB_DEV uint64_t block_exscan_u64(uint64_t v, uint64_t* red, uint64_t* total) {
+// Exclusive block scans of two uint64 values in thread order, one pair of barriers;
+// returns this thread's prefixes and the block totals.
+AB_DEV void block_exscan2_u64(uint64_t v0, uint64_t v1, uint64_t* red0, uint64_t* red1,
+                              uint64_t& before0, uint64_t& before1, uint64_t& total0,
+                              uint64_t& total1) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  uint64_t inc = v;
+  uint64_t inc0 = v0, inc1 = v1;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (l >= o) inc += y;
+    const uint64_t y0 = __shfl_up_sync(0xffffffffu, inc0, o);
+    const uint64_t y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+    if (l >= o) {
+      inc0 += y0;
+      inc1 += y1;
+    }
   }
   __syncthreads();
-  if (l == 31) red[w] = inc;
+  if (l == 31) {
+    red0[w] = inc0;
+    red1[w] = inc1;
+  }
   __syncthreads();
-  uint64_t before = 0, tot = 0;
+  uint64_t b0 = 0, b1 = 0, t0 = 0, t1 = 0;
 #pragma unroll
   for (int i = 0; i < PLAN_WARPS; ++i) {
-    if (i < w) before += red[i];
-    tot += red[i];
+    if (i < w) {
+      b0 += red0[i];
+      b1 += red1[i];
+    }
+    t0 += red0[i];
+    t1 += red1[i];
   }
-  *total = tot;
-  return before + inc - v;
+  before0 = b0 + inc0 - v0;
+  before1 = b1 + inc1 - v1;
+  total0 = t0;
+  total1 = t1;
 }
 
 template <bool STAGED>
@@ -140,19 +164,55 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   const float* grow = a.S + (size_t)row * nK;
   const float* srow = grow;
   const int nK4 = (nK + 3) >> 2;  // staged row padded with zeros to whole float4s
-  if (STAGED) {
-    for (int j = tid; j < nK4 * 4; j += PLAN_THREADS) srow_smem[j] = (j < nK) ? __ldg(grow + j) : 0.f;
-    __syncthreads();
-    srow = srow_smem;
-  }
   const uint64_t s = (uint64_t)a.s;
   const uint64_t target = s * TWO32;
 
+  // ---- positive blocks and their total score (fewer than s positive blocks = budget
+  // unreachable); per-thread sums in compensated fp32, block sum in fp64.  With the row
+  // staged in shared memory this pass also copies it there.
+  uint64_t npos = 0;
+  double tot = 0.0;
+  {
+    float sum = 0.f, comp = 0.f;
+    auto acc = [&](float sv) {
+      if (sv > 0.f) {
+        const float y = sv - comp, t2 = sum + y;
+        comp = (t2 - sum) - y;
+        sum = t2;
+        ++npos;
+      }
+    };
+    if (STAGED) {
+      const bool vec = ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
+      float4* s4 = reinterpret_cast<float4*>(srow_smem);
+      for (int j = tid; j < nK4; j += PLAN_THREADS) {
+        float4 v;
+        if (vec) {
+          v = __ldg(reinterpret_cast<const float4*>(grow) + j);
+        } else {
+          v.x = (4 * j < nK) ? __ldg(grow + 4 * j) : 0.f;
+          v.y = (4 * j + 1 < nK) ? __ldg(grow + 4 * j + 1) : 0.f;
+          v.z = (4 * j + 2 < nK) ? __ldg(grow + 4 * j + 2) : 0.f;
+          v.w = (4 * j + 3 < nK) ? __ldg(grow + 4 * j + 3) : 0.f;
+        }
+        s4[j] = v;
+        acc(v.x);
+        acc(v.y);
+        acc(v.z);
+        acc(v.w);
+      }
+      srow = srow_smem;  // read only after the barriers of the block sum below
+    } else {
+      for (int j = tid; j < nK; j += PLAN_THREADS) acc(__ldg(grow + j));
+    }
+    tot = (double)sum - (double)comp;
+  }
+  block_sum_cd(npos, tot, red, redd);
+  const bool reachable = npos >= s;
+
   // ---- lambda*: the smallest positive fp32 (bit pattern in (0, 0x7F800000]) with
   // F(lambda) >= s 2^32.  F is monotone in the bit pattern, so any search that brackets
-  // the boundary and bisects finds the same lambda as a full 31-step bisection.  A
-  // water-filling estimate lambda <- (s - |saturated|) / (sum of the unsaturated S)
-  // starts the search a few ulps from the boundary.
+  // the boundary and bisects finds the same lambda as a full 31-step bisection.
   auto F = [&](uint32_t bits) -> uint64_t {
     const float lam = __uint_as_float(bits);
     uint64_t part = 0;
@@ -160,37 +220,21 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       const float4* s4 = reinterpret_cast<const float4*>(srow);
       for (int j = tid; j < nK4; j += PLAN_THREADS) {
         const float4 v = s4[j];
-        part += fixed_q(lam, v.x) + fixed_q(lam, v.y) + fixed_q(lam, v.z) + fixed_q(lam, v.w);
+        add_q(lam, v.x, part);
+        add_q(lam, v.y, part);
+        add_q(lam, v.z, part);
+        add_q(lam, v.w, part);
       }
     } else {
-      for (int j = tid; j < nK; j += PLAN_THREADS) part += fixed_q(lam, srow[j]);
+      for (int j = tid; j < nK; j += PLAN_THREADS) add_q(lam, srow[j], part);
     }
     return block_sum_u64(part, red);
   };
   uint32_t lo = 0u, hi = 0x7F800000u;
-  // positive blocks and their total score; fewer than s positive blocks = budget unreachable
-  // per-thread sums in compensated fp32 (no per-element fp64 conversions), block sum in fp64
-  uint64_t npos = 0;
-  double tot = 0.0;
-  {
-    float sum = 0.f, comp = 0.f;
-    for (int j = tid; j < nK; j += PLAN_THREADS) {
-      const float sv = srow[j];
-      if (sv > 0.f) {
-        const float y = sv - comp, t2 = sum + y;
-        comp = (t2 - sum) - y;
-        sum = t2;
-        ++npos;
-      }
-    }
-    tot = (double)sum - (double)comp;
-  }
-  block_sum_cd(npos, tot, red, redd);
-  const bool reachable = npos >= s;
   if (reachable) {
     // Water filling in fp64 (a starting point only): lambda <- (s - |saturated|) / (sum of
-    // the unsaturated scores) until the saturated set stops growing; in practice a few
-    // rounds, ending within an ulp or two of lambda*.
+    // the unsaturated scores) until the saturated set stops growing; in practice one or
+    // two rounds, ending within an ulp or two of lambda*.
     double lam_w = (tot > 0.0) ? (double)a.s / tot : 0.0;
     double rest_est = tot;
     for (int it = 0; it < 32 && lam_w > 0.0; ++it) {
@@ -269,94 +313,73 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
 
   // ---- per element code on this thread's contiguous chunk: the fixed-point q_j (< 2^32 - 255)
   // or SAT for an inclusion probability of exactly 1 (when the budget is unreachable: every
-  // positive block is SAT and zero blocks have code 0).  With the row staged in shared
-  // memory the codes overwrite the thread's own slots, so the two selection passes below
-  // are integer-only.
+  // positive block is SAT and the others have code 0).  With the row staged in shared
+  // memory the codes overwrite the thread's own slots: every read of the scores by the
+  // other threads happened before the barriers of the last block sum.
   constexpr uint32_t SAT = 0xFFFFFFFFu;
   uint32_t* code_smem = reinterpret_cast<uint32_t*>(srow_smem);
   auto code_from_score = [&](float sv) -> uint32_t {
     if (reachable) {
-      const uint64_t q = fixed_q(lam, sv);
-      return q == TWO32 ? SAT : (uint32_t)q;
+      uint32_t q;
+      return fixed_q32(lam, sv, q) ? SAT : q;
     }
     return (sv > 0.f) ? SAT : 0u;
   };
-  auto code_of = [&](int j) -> uint32_t {
-    if (STAGED) return code_smem[j];
-    return code_from_score(srow[j]);
-  };
   const int per = (nK + PLAN_THREADS - 1) / PLAN_THREADS;
   const int j0 = min(nK, tid * per), j1 = min(nK, j0 + per);
-  uint64_t my_sat = 0, my_rest = 0, my_zero = 0;
+  // my_rest: the chunk's total q (budget reachable) or its number of code-0 blocks
+  uint64_t my_sat = 0, my_rest = 0;
   for (int j = j0; j < j1; ++j) {
     const uint32_t c = code_from_score(srow[j]);
-    if (STAGED) code_smem[j] = c;  // own slot; every read of the scores happened before
+    if (STAGED) code_smem[j] = c;
     if (c == SAT) ++my_sat;
-    else if (reachable) my_rest += c;
-    else ++my_zero;
+    else my_rest += reachable ? c : 1u;
   }
-  uint64_t n_sat = 0, tot_rest = 0, n_zero_tot = 0;
-  const uint64_t sat_before = block_exscan_u64(my_sat, red, &n_sat);
-  const uint64_t rest_before = block_exscan_u64(my_rest, red2, &tot_rest);
-  uint64_t zero_before = 0;
-  if (!reachable) zero_before = block_exscan_u64(my_zero, red, &n_zero_tot);
+  uint64_t sat_before, rest_before, n_sat, tot_rest;
+  block_exscan2_u64(my_sat, my_rest, red, red2, sat_before, rest_before, n_sat, tot_rest);
 
   const uint32_t U = philox4x32_10_w0((uint32_t)row, (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
                                       0u, (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
-  // lattice points U + k 2^32 below x (x <= s 2^32, so at most s)
-  auto below = [&](uint64_t x) -> uint64_t { return x > U ? ((x - U - 1) >> 32) + 1 : 0ull; };
+  // lattice points U + k 2^32 below x, for 0 <= x <= s 2^32 (U < 2^32)
+  const uint64_t CB = TWO32 - 1u - (uint64_t)U;
+  auto below = [&](uint64_t x) -> uint64_t { return (x + CB) >> 32; };
   // Saturated blocks come first in the layout, block k of them covering [k 2^32, (k+1) 2^32):
-  // each holds exactly one lattice point, so every saturated block is drawn.
-
-  // ---- selection flags, counted per chunk
-  uint64_t my_sel = 0;
-  {
-    uint64_t pos = n_sat * TWO32 + rest_before, zero_i = zero_before;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t c = code_of(j);
-      bool sel;
-      if (c == SAT) {
-        sel = true;
-      } else if (reachable) {
-        const uint64_t st = min(pos, target), en = min(pos + c, target);
-        sel = below(en) > below(st);
-        pos += c;
-      } else {
-        sel = zero_i++ < s - n_sat;
-      }
-      my_sel += sel;
-    }
-  }
-  uint64_t n_sel = 0;
-  const uint64_t out_before = block_exscan_u64(my_sel, red, &n_sel);
+  // each holds exactly one lattice point, so every saturated block is drawn.  The other
+  // blocks follow in ascending order; this thread's chunk covers [start, start + my_rest).
+  // With the budget unreachable, the first s - n_sat code-0 blocks (in order) complete it.
+  const uint64_t start = n_sat * TWO32 + rest_before;
+  const uint64_t need = s - min(n_sat, s);
+  const uint64_t my_sel =
+      my_sat + (reachable ? below(min(start + my_rest, target)) - below(min(start, target))
+                          : (rest_before < need ? min(my_rest, need - rest_before) : 0ull));
+  uint64_t out_before, zero_b, n_sel, zero_t;
+  block_exscan2_u64(my_sel, 0ull, red, red2, out_before, zero_b, n_sel, zero_t);
   if (n_sel != s && tid == 0) ab_flag(AB_ERR_DEVICE_CHECK);  // cannot happen; guards the writes
 
-  // ---- write ascending idx and log(pi)
+  // ---- write ascending idx and the fixed-point probability (its log follows below)
   {
-    uint64_t pos = n_sat * TWO32 + rest_before, zero_i = zero_before;
+    uint64_t pos = start, zero_i = rest_before;
     uint64_t o = out_before;
     int32_t* oidx = a.idx + (size_t)row * a.s;
-    float* olp = a.logpi + (size_t)row * a.s;
+    uint32_t* oraw = reinterpret_cast<uint32_t*>(a.logpi + (size_t)row * a.s);
     for (int j = j0; j < j1; ++j) {
-      const uint32_t c = code_of(j);
+      const uint32_t c = STAGED ? code_smem[j] : code_from_score(srow[j]);
       bool sel;
-      uint64_t qq = TWO32;
+      uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
       if (c == SAT) {
         sel = true;
       } else if (reachable) {
         const uint64_t st = min(pos, target), en = min(pos + c, target);
-        sel = below(en) > below(st);
-        qq = en - st;
+        sel = below(en) != below(st);
+        qq = (uint32_t)(en - st);
         pos += c;
       } else {
-        sel = zero_i++ < s - n_sat;
+        sel = zero_i++ < need;
       }
       if (sel) {
         if (o < s) {
           oidx[o] = j;
-          // the probability's fixed-point value for now (2^32 - 1 stands for pi = 1: a capped
-          // or ordinary q is at most 2^32 - 256); its log follows in a compacted pass
-          reinterpret_cast<uint32_t*>(olp)[o] = (qq == TWO32) ? 0xFFFFFFFFu : (uint32_t)qq;
+          oraw[o] = qq;
         }
         ++o;
       }
