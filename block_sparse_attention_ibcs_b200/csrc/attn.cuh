@@ -23,20 +23,18 @@
 //                                       shift tile b_t, from shared memory)
 //              O += P_t V_t            (M=128, N=d, K=128; A = P from tensor memory, B = V
 //                                       read MN-major from the same tile layout)
-//              l += P_t 1              (M=128, N=16, K=128; the same A, B = a tile of bf16
-//                                       ones: the row sums of the bf16 weights PV used)
 //   warps 0-3  softmax: thread r owns query row r = TMEM lane r.  Loads its Q row into
 //              tensor memory once, then per tile reads S (already shifted), keeps a lazy
 //              online max (raised only when a tile exceeds it by more than 2^8, decided
-//              per warp), writes P as bf16 into tensor memory, rescales its O row and l
-//              when the max moved, and finally writes O / l.
+//              per warp), writes P as bf16 into tensor memory, rescales its O row when
+//              the max moved, and finally writes O / l.
 // The shift -log(pi_j) of a sampled block (in logit units: -log(pi_j) * sqrt(d)) enters
 // through the tensor cores as one more K=16 step: A = [1 1 0 ... 0] for every query row,
 // B row n = [hi_n lo_n 0 ... 0] with hi = bf16(shift), lo = bf16(shift - hi), so S gains
 // hi + lo (the shift to about 2^-17 relative) and the softmax threads touch no shared
 // memory per tile.  Padding and out-of-range rows get hi = -2^100: their weight is 0.
 // Tensor memory: S [0,128), O [128,128+d), P0 [256,320), P1 [320,384), Q [384,384+d/2),
-// ones [448,464), l [464,480).  All waits are bounded; a stuck pipeline records AB_ERR_DEVICE_TIMEOUT
+// ones [448,464).  All waits are bounded; a stuck pipeline records AB_ERR_DEVICE_TIMEOUT
 // and every role drains and exits.
 #pragma once
 
@@ -89,9 +87,7 @@ struct AttnSmem {
   static constexpr uint32_t SHIFT_OFF = 0;                                  // ATTN_STAGES
   static constexpr uint32_t K_OFF = SHIFT_OFF + ATTN_STAGES * SHIFT_BYTES;  // ATTN_STAGES
   static constexpr uint32_t V_OFF = K_OFF + ATTN_STAGES * TILE_BYTES;       // ATTN_STAGES
-  static constexpr uint32_t ONES_OFF = V_OFF + ATTN_STAGES * TILE_BYTES;    // 4 KB of bf16 1.0
-  static constexpr uint32_t ONES_BYTES = 4096u;
-  static constexpr uint32_t BAR_OFF = ONES_OFF + ONES_BYTES;
+  static constexpr uint32_t BAR_OFF = V_OFF + ATTN_STAGES * TILE_BYTES;
   static constexpr uint32_t NBARS = 17;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBARS * 8u;
   static constexpr uint32_t BYTES = MISC_OFF + 16u;
@@ -148,12 +144,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     mbar_init(&bars[B_DRAIN], 1);
     fence_mbar_init();
   }
-  // zero the shift tiles once (per tile only the first 4 bytes of each row change) and
-  // fill the ones tile of the row-sum MMA
+  // zero the shift tiles once: per tile only the first 4 bytes of each row change
   for (uint32_t o = tid * 16u; o < ATTN_STAGES * L::SHIFT_BYTES; o += ATTN_THREADS * 16u)
     *(uint4*)(smem + L::SHIFT_OFF + o) = make_uint4(0u, 0u, 0u, 0u);
-  for (uint32_t o = tid * 16u; o < L::ONES_BYTES; o += ATTN_THREADS * 16u)
-    *(uint4*)(smem + L::ONES_OFF + o) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   fence_proxy_async_smem();
   if (warp == 11) {
     tmem_alloc(tmem_slot, 512);
@@ -169,7 +162,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
   const uint32_t TM_P1 = tmem + 320;    // columns [320,384)
   const uint32_t TM_Q = tmem + 384;     // columns [384, 384+D/2): the Q row as bf16 pairs
   const uint32_t TM_ONES = tmem + 448;  // columns [448,464): A of the shift step
-  const uint32_t TM_L = tmem + 464;     // columns [464,480): row sums of P (column 464 used)
 
   if (warp >= 4 && warp < 11) {
     // ================================================================ producers
@@ -319,14 +311,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
-      constexpr uint32_t IDESC_L = idesc_bf16_f32(128, 16, 0, 0);
       // base descriptors; per 16-element K step only the start-address field moves
       // (stage b adds b * TILE_BYTES / 16 to the start-address field)
       const uint64_t dk0 = sdesc_sw128(sbase + L::K_OFF, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sbase + L::V_OFF, L::CHUNK_BYTES, 1024);
       const uint64_t db0 = sdesc_noswizzle(sbase + L::SHIFT_OFF, L::SHIFT_KHALF, 128);
-      // all-ones B (16 x 16 per step): any layout reads ones; lbo/sbo keep it within 512 B
-      const uint64_t d1 = sdesc_noswizzle(sbase + L::ONES_OFF, 128, 256);
       bool ok = mbar_wait(&bars[B_QFULL], 0, abort_flag, a.timeout_ns);
       tc_fence_after();
       int nqk = 0, npv = 0;              // next QK / PV to issue (npv < nqk)
@@ -343,9 +332,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           for (int kk = 0; kk < 8; ++kk)  // 16 keys per MMA: 8 TMEM columns of P, 2 KB of V
             umma_f16_ts(TM_O, ap + kk * 8, dv0 + (uint64_t)((sp * L::TILE_BYTES + kk * 2048) >> 4), IDESC_PV,
                         (npv > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_f16_ts(TM_L, ap + kk * 8, d1, IDESC_L, (npv > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bars[B_PVDONE0 + (npv & 1)]);
           umma_commit(&bars[B_EMPTY0 + sp]);
           ev(EV_PV, npv);
@@ -392,6 +378,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c = a.scale_log2;
     float m_run = -INFINITY;  // reference max (log2 domain)
+    float l_run = 0.f;
     bool ok = true;
     {  // Q row r (zeros past the sequence end) and the ones of the shift step -> TMEM
       const uint4* qrow = (const uint4*)(a.Q + head_off + (size_t)(row0 + min(r, nvalid - 1)) * D);
@@ -436,14 +423,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       const float* z = reinterpret_cast<const float*>(zr);
       float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmax3(z[k], z[8 + k], z[16 + k]);
+      for (int k = 0; k < 8; ++k) mx[k] = z[k];
 #pragma unroll
-      for (int k = 24; k < 120; k += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], z[k + i], z[k + 8 + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[120 + i]);
-      float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
+      for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], z[k]);
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
       if (mt < PAD_LOGIT_LOG2) mt = -INFINITY;  // every column of the tile is padding
       // Lazy rescale, decided per warp: tcgen05.ld/st are warp-collective, so when any
       // row of the warp has to raise its reference max, every row of the warp moves to
@@ -468,19 +452,28 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       }
       if (r == 0) ev(EV_SM_PBUF, t);
       const uint32_t padr = (st ? TM_P1 : TM_P0) + lane_off;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(nmref, nmref);
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {  // 32 keys -> 16 TMEM columns of packed bf16 pairs
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c0 = 32 * g + 2 * e;
-          const float2 x = __ffma2_rn(make_float2(z[c0], z[c0 + 1]), c2, nm2);  // paired fp32 FMA
-          pk[e] = pack_bf16x2_rn(fast_exp2(x.x), fast_exp2(x.y));
+          const float x0 = fmaf(z[c0], c, nmref);
+          const float x1 = fmaf(z[c0 + 1], c, nmref);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          ls[(2 * e) & 7] += p0;
+          ls[(2 * e + 1) & 7] += p1;
+          pk[e] = pack_bf16x2_rn(p0, p1);
         }
         tmem_st_32x32b_x16(padr + 16 * g, pk);
       }
-      if (rescale && t > 0) {  // warp-uniform; O and l hold no data before PV(0)
+      const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      l_run = l_run * alpha + lsum;
+      if (rescale && t > 0) {  // warp-uniform; O holds no data before PV(0)
         // O is stable once PV(t-1) has completed
         ok = mbar_wait(&bars[B_PVDONE0 + (st ^ 1)], ((t - 1) >> 1) & 1, abort_flag, a.timeout_ns);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -494,10 +487,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
           tmem_st_32x32b_x32(TM_O + lane_off + c0, v);
         }
-        uint32_t lv;
-        tmem_ld_32x32b_x1(TM_L + lane_off, lv);
-        tmem_wait_ld();
-        tmem_st_32x32b_x1(TM_L + lane_off, __float_as_uint(__uint_as_float(lv) * alpha));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -509,10 +498,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      uint32_t lv;
-      tmem_ld_32x32b_x1(TM_L + lane_off, lv);
-      tmem_wait_ld();
-      const float l_run = __uint_as_float(lv);
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       uint16_t* orow = a.O + head_off + (size_t)(row0 + r) * D;
 #pragma unroll
