@@ -18,13 +18,15 @@ import os
 
 __all__ = [
     "ABError", "ABParams", "params", "lib", "ab_workspace_bytes", "ab_select",
-    "ab_select_debug", "ab_plan", "ab_sample", "ab_attn", "ab_attn_dense", "ab_get_status",
-    "ab_status_string", "ab_version", "LIB_PATH",
+    "ab_select_debug", "ab_plan", "ab_plan_variant", "ab_sample", "ab_attn", "ab_attn_dense",
+    "ab_get_status", "ab_status_string", "ab_version", "LIB_PATH", "PLAN_MODES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libabattn.so")
 
 AB_OK = 0
+# ab_plan_mode (include/abattn.h): planner variants for the page's ablations
+PLAN_MODES = {"sip": 0, "sip_no_ipw": 1, "uniform": 2, "topk": 3}
 STATUS_NAMES = {
     0: "AB_OK", -1: "AB_ERR_INVALID_ARG", -2: "AB_ERR_UNSUPPORTED", -3: "AB_ERR_CUDA",
     -4: "AB_ERR_DEVICE_TIMEOUT", -5: "AB_ERR_WORKSPACE", -6: "AB_ERR_NOT_IMPLEMENTED",
@@ -56,6 +58,7 @@ _SIGS = {
     "ab_select": [_P, _vp, _vp, _vp, _vp, _sz, _vp],
     "ab_select_debug": [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp],
     "ab_plan": [_P, _vp, _i, _u64, _u64, _vp, _vp, _vp],
+    "ab_plan_variant": [_P, _vp, _i, _u64, _u64, _i, _vp, _vp, _vp],
     "ab_sample": [_P, _vp, _i, _u64, _u64, _vp, _vp, _vp],
     "ab_attn": [_P, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp],
     "ab_attn_dense": [_P, _vp, _vp, _vp, _vp, _vp],
@@ -145,6 +148,18 @@ def ab_plan(p, S, s, seed, offset, idx, logpi, stream=None):
     _check(lib().ab_plan(ctypes.byref(p), _ptr(S, "S", torch.float32), int(s), int(seed), int(offset),
                          _ptr(idx, "idx", torch.int32), _ptr(logpi, "logpi", torch.float32),
                          _stream(stream)), "ab_plan")
+
+
+def ab_plan_variant(p, S, s, seed, offset, mode, idx, logpi, stream=None):
+    """Planner variant ``mode`` (a name in PLAN_MODES or its number); S may be None for
+    "uniform"."""
+    import torch
+
+    m = PLAN_MODES[mode] if isinstance(mode, str) else int(mode)
+    _check(lib().ab_plan_variant(ctypes.byref(p), _ptr(S, "S", torch.float32), int(s), int(seed),
+                                 int(offset), m, _ptr(idx, "idx", torch.int32),
+                                 _ptr(logpi, "logpi", torch.float32), _stream(stream)),
+           "ab_plan_variant")
 
 
 def ab_sample(p, pi, s, seed, offset, idx, logpi, stream=None):

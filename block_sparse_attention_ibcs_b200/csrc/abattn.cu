@@ -123,7 +123,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
 }
 
 ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t offset,
-                   int32_t* idx, float* logpi, cudaStream_t st) {
+                   int mode, int32_t* idx, float* logpi, cudaStream_t st) {
   PlanArgs a;
   a.S = S;
   a.idx = idx;
@@ -132,7 +132,20 @@ ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t
   a.s = s;
   a.seed = seed;
   a.offset = offset;
+  a.mode = mode;
   const unsigned rows = (unsigned)(d.BH * d.nQ);
+  if (mode == AB_PLAN_TOPK) {
+    if (d.nK <= PLAN_SMEM_MAX_FLOATS) {
+      const size_t smem = (size_t)d.nK * 4;  // the row's keys
+      if (cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PLAN_SMEM_MAX_FLOATS * 4) != cudaSuccess)
+        return launch_status();
+      topk_kernel<true><<<rows, PLAN_THREADS, smem, st>>>(a);
+    } else {
+      topk_kernel<false><<<rows, PLAN_THREADS, 0, st>>>(a);
+    }
+    return launch_status();
+  }
   if (d.nK <= PLAN_SMEM_MAX_FLOATS) {
     const size_t smem = (size_t)((d.nK + 3) / 4) * 16;  // row padded to whole float4s
     // per-device attribute; cheap enough to set on every launch
@@ -240,14 +253,15 @@ ab_status select_common(const ab_params* p, const void* Q, const void* K, float*
 }
 
 ab_status plan_common(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
-                      int32_t* idx, float* logpi, void* stream) {
+                      int mode, int32_t* idx, float* logpi, void* stream) {
   Dims d;
   ab_status r = check_params(p, &d);
   if (r != AB_OK) return r;
-  if (!S || !idx || !logpi || ((uintptr_t)S & 3) || ((uintptr_t)idx & 3) || ((uintptr_t)logpi & 3))
-    return AB_ERR_INVALID_ARG;
+  if (mode < AB_PLAN_SIP || mode > AB_PLAN_TOPK) return AB_ERR_INVALID_ARG;
+  if (mode != AB_PLAN_UNIFORM && (!S || ((uintptr_t)S & 3))) return AB_ERR_INVALID_ARG;
+  if (!idx || !logpi || ((uintptr_t)idx & 3) || ((uintptr_t)logpi & 3)) return AB_ERR_INVALID_ARG;
   if (s < 1 || s > d.nK) return AB_ERR_INVALID_ARG;
-  return run_plan(d, S, s, seed, offset, idx, logpi, (cudaStream_t)stream);
+  return run_plan(d, S, s, seed, offset, mode, idx, logpi, (cudaStream_t)stream);
 }
 
 }  // namespace
@@ -276,12 +290,17 @@ ab_status ab_select_debug(const ab_params* p, const void* Q, const void* K, floa
 
 ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
                   int32_t* idx, float* logpi, void* stream) {
-  return plan_common(p, S, s, seed, offset, idx, logpi, stream);
+  return plan_common(p, S, s, seed, offset, AB_PLAN_SIP, idx, logpi, stream);
+}
+
+ab_status ab_plan_variant(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
+                          int mode, int32_t* idx, float* logpi, void* stream) {
+  return plan_common(p, S, s, seed, offset, mode, idx, logpi, stream);
 }
 
 ab_status ab_sample(const ab_params* p, const float* pi, int s, uint64_t seed, uint64_t offset,
                     int32_t* idx, float* logpi, void* stream) {
-  return plan_common(p, pi, s, seed, offset, idx, logpi, stream);
+  return plan_common(p, pi, s, seed, offset, AB_PLAN_SIP, idx, logpi, stream);
 }
 
 ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* V,

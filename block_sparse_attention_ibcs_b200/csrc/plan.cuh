@@ -36,11 +36,12 @@ constexpr int PLAN_SMEM_MAX_FLOATS = 40 * 1024;  // 160 KB of staged row
 constexpr uint64_t TWO32 = 1ull << 32;
 
 struct PlanArgs {
-  const float* S;   // [rows, nK]
+  const float* S;   // [rows, nK] (not read in the uniform variant)
   int32_t* idx;     // [rows, s]
   float* logpi;     // [rows, s]
   int nK, s;
   uint64_t seed, offset;
+  int mode;         // ab_plan_mode: SIP, SIP without inverse-probability weights, uniform
 };
 
 // Philox4x32-10 (Salmon et al., SC'11), word 0 of the output block.
@@ -163,6 +164,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   const int nK = a.nK;
   const float* grow = a.S + (size_t)row * nK;
   const float* srow = grow;
+  const bool uniform = a.mode == AB_PLAN_UNIFORM;
+  // score j of the row when it is not staged (the uniform variant reads no scores)
+  auto sv_at = [&](int j) -> float { return uniform ? 1.f : __ldg(grow + j); };
   const int nK4 = (nK + 3) >> 2;  // staged row padded with zeros to whole float4s
   const uint64_t s = (uint64_t)a.s;
   const uint64_t target = s * TWO32;
@@ -187,7 +191,12 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       float4* s4 = reinterpret_cast<float4*>(srow_smem);
       for (int j = tid; j < nK4; j += PLAN_THREADS) {
         float4 v;
-        if (vec) {
+        if (uniform) {  // the same score for every block
+          v.x = (4 * j < nK) ? 1.f : 0.f;
+          v.y = (4 * j + 1 < nK) ? 1.f : 0.f;
+          v.z = (4 * j + 2 < nK) ? 1.f : 0.f;
+          v.w = (4 * j + 3 < nK) ? 1.f : 0.f;
+        } else if (vec) {
           v = __ldg(reinterpret_cast<const float4*>(grow) + j);
         } else {
           v.x = (4 * j < nK) ? __ldg(grow + 4 * j) : 0.f;
@@ -203,7 +212,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       }
       srow = srow_smem;  // read only after the barriers of the block sum below
     } else {
-      for (int j = tid; j < nK; j += PLAN_THREADS) acc(__ldg(grow + j));
+      for (int j = tid; j < nK; j += PLAN_THREADS) acc(sv_at(j));
     }
     tot = (double)sum - (double)comp;
   }
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         add_q(lam, v.w, part);
       }
     } else {
-      for (int j = tid; j < nK; j += PLAN_THREADS) add_q(lam, srow[j], part);
+      for (int j = tid; j < nK; j += PLAN_THREADS) add_q(lam, sv_at(j), part);
     }
     return block_sum_u64(part, red);
   };
@@ -244,7 +253,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       {
         float sum = 0.f, comp = 0.f;
         for (int j = tid; j < nK; j += PLAN_THREADS) {
-          const float sv = srow[j];
+          const float sv = STAGED ? srow[j] : sv_at(j);
           if (sv > 0.f) {
             if (__fmul_rn(lw, sv) >= 1.f) {
               ++nsat;
@@ -330,7 +339,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   // my_rest: the chunk's total q (budget reachable) or its number of code-0 blocks
   uint64_t my_sat = 0, my_rest = 0;
   for (int j = j0; j < j1; ++j) {
-    const uint32_t c = code_from_score(srow[j]);
+    const uint32_t c = code_from_score(STAGED ? srow[j] : sv_at(j));
     if (STAGED) code_smem[j] = c;
     if (c == SAT) ++my_sat;
     else my_rest += reachable ? c : 1u;
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     int32_t* oidx = a.idx + (size_t)row * a.s;
     uint32_t* oraw = reinterpret_cast<uint32_t*>(a.logpi + (size_t)row * a.s);
     for (int j = j0; j < j1; ++j) {
-      const uint32_t c = STAGED ? code_smem[j] : code_from_score(srow[j]);
+      const uint32_t c = STAGED ? code_smem[j] : code_from_score(sv_at(j));
       bool sel;
       uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
       if (c == SAT) {
@@ -392,7 +401,118 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     uint32_t* raw = reinterpret_cast<uint32_t*>(olp);
     for (int o = tid; o < a.s; o += PLAN_THREADS) {
       const uint32_t q = raw[o];
-      olp[o] = (q == 0xFFFFFFFFu) ? 0.f : (float)log((double)q * (1.0 / 4294967296.0));
+      olp[o] = (q == 0xFFFFFFFFu || a.mode == AB_PLAN_SIP_NO_IPW)
+                   ? 0.f
+                   : (float)log((double)q * (1.0 / 4294967296.0));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- top-k
+//
+// Top-k variant of the planner (AB-Attention page, ablations: the deterministic top-k
+// selection SIP is compared against): per row, the s blocks with the largest scores, ties
+// to the lower block index, ascending; log pi = 0 (pi = 1 for every kept block, no
+// reweighting).  Scores are ranked by an order-preserving 32-bit key (score_key: larger
+// score, larger key; +0 above -0; NaN below every number).  A 4-pass radix select (8-bit
+// digits from the top) finds the key K* of the s-th largest; every key > K* is kept, plus
+// the first s - |{key > K*}| keys equal to K* in block order.
+
+AB_DEV uint32_t score_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  if (v != v) return 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+template <bool STAGED>
+__global__ void __launch_bounds__(PLAN_THREADS) topk_kernel(PlanArgs a) {
+  extern __shared__ uint32_t key_smem[];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t sel_digit, sel_above;
+  __shared__ uint64_t red[PLAN_WARPS];
+  __shared__ uint64_t red2[PLAN_WARPS];
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int nK = a.nK;
+  const float* grow = a.S + (size_t)row * nK;
+  auto key_at = [&](int j) -> uint32_t { return STAGED ? key_smem[j] : score_key(__ldg(grow + j)); };
+  if (STAGED) {
+    for (int j = tid; j < nK; j += PLAN_THREADS) key_smem[j] = score_key(__ldg(grow + j));
+  }
+  uint32_t prefix = 0u, mask = 0u;
+  uint32_t remaining = (uint32_t)a.s;  // rank of K* among the keys matching the prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += PLAN_THREADS) hist[b] = 0u;
+    __syncthreads();  // also orders the staging above before the first histogram
+    for (int j = tid; j < nK; j += PLAN_THREADS) {
+      const uint32_t k = key_at(j);
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns digits 255 - 8l down to 248 - 8l; find the digit where the count of
+      // keys at or above it first reaches `remaining`
+      uint32_t own = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) own += hist[255 - 8 * tid - i];
+      uint32_t inc = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (tid >= o) inc += y;
+      }
+      const uint32_t before = inc - own;  // keys in higher digits of the lanes before
+      const bool mine = before < remaining && inc >= remaining;
+      if (mine) {
+        uint32_t above = before;
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t dgt = 255u - 8u * tid - i;
+          const uint32_t c = hist[dgt];
+          if (above + c >= remaining) {
+            sel_digit = dgt;
+            sel_above = above;
+            break;
+          }
+          above += c;
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= sel_digit << shift;
+    mask |= 255u << shift;
+    remaining -= sel_above;
+    __syncthreads();  // sel_digit / sel_above are rewritten by the next pass
+  }
+  const uint32_t kstar = prefix;
+  const uint64_t need_eq = remaining;  // keys equal to K* to keep (>= 1)
+
+  // keep every key > K* and the first need_eq keys == K*; contiguous chunks keep block order
+  const int per = (nK + PLAN_THREADS - 1) / PLAN_THREADS;
+  const int j0 = min(nK, tid * per), j1 = min(nK, j0 + per);
+  uint64_t my_gt = 0, my_eq = 0;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t k = key_at(j);
+    my_gt += k > kstar;
+    my_eq += k == kstar;
+  }
+  uint64_t gt_before, eq_before, n_gt, n_eq;
+  block_exscan2_u64(my_gt, my_eq, red, red2, gt_before, eq_before, n_gt, n_eq);
+  const uint64_t my_sel = my_gt + (eq_before < need_eq ? min(my_eq, need_eq - eq_before) : 0ull);
+  uint64_t out_before, zb, n_sel, zt;
+  block_exscan2_u64(my_sel, 0ull, red, red2, out_before, zb, n_sel, zt);
+  if (n_sel != (uint64_t)a.s && tid == 0) ab_flag(AB_ERR_DEVICE_CHECK);  // cannot happen
+  uint64_t o = out_before, eq_i = eq_before;
+  int32_t* oidx = a.idx + (size_t)row * a.s;
+  float* olp = a.logpi + (size_t)row * a.s;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t k = key_at(j);
+    const bool sel = k > kstar || (k == kstar && eq_i++ < need_eq);
+    if (sel) {
+      if (o < (uint64_t)a.s) {
+        oidx[o] = j;
+        olp[o] = 0.f;
+      }
+      ++o;
     }
   }
 }

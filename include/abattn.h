@@ -114,6 +114,28 @@ ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint
 ab_status ab_sample(const ab_params* p, const float* pi, int s, uint64_t seed,
                     uint64_t offset, int32_t* idx, float* logpi, void* stream);
 
+/* Planner variants for the ablations on the AB-Attention page (the selection rules SIP
+ * is compared against).  Same arguments and output layout as ab_plan, plus `mode`:
+ *   AB_PLAN_SIP         exactly ab_plan.
+ *   AB_PLAN_SIP_NO_IPW  the same draw as ab_plan, but logpi = 0 for every block: the
+ *                       sampled blocks enter attention without inverse-probability
+ *                       reweighting.
+ *   AB_PLAN_UNIFORM     ab_plan's fixed-point inclusion probabilities and systematic
+ *                       draw on a constant score row (S is not read): pi_j = s / nK up
+ *                       to the 2^-32 fixed point and the trimmed tail; logpi as ab_plan.
+ *   AB_PLAN_TOPK        the s blocks with the largest S (deterministic; ties to the lower
+ *                       block index; NaN ranks below every number, +0 above -0), logpi =
+ *                       0; seed and offset are unused.
+ * Returns AB_ERR_INVALID_ARG for an unknown mode.                                      */
+typedef enum {
+  AB_PLAN_SIP = 0,
+  AB_PLAN_SIP_NO_IPW = 1,
+  AB_PLAN_UNIFORM = 2,
+  AB_PLAN_TOPK = 3
+} ab_plan_mode;
+ab_status ab_plan_variant(const ab_params* p, const float* S, int s, uint64_t seed,
+                          uint64_t offset, int mode, int32_t* idx, float* logpi, void* stream);
+
 /* Packed-tile sparse attention ("premises & limits" section of the AB-Attention page).
  * For each query q of query block i:
  *   O_q = sum_{j in idx, t in block j, t < N} e^{z_t} v_t / sum e^{z_t},

@@ -18,7 +18,9 @@ Every step follows the AB-Attention page (onedev.kr/papers/1521):
            small blocks gathered by index into full tiles; −log π shift, online
            softmax and value accumulation in one pass; no token reordering.
 * [ABL]    ablation paragraph: position-based 16-query segment means (used here
-           as the k-means initialisation, and alone when kmeans_iters = 0).
+           as the k-means initialisation, and alone when kmeans_iters = 0), and
+           the selection rules SIP is compared against: deterministic top-k,
+           sampling without inverse-probability weighting, uniform sampling.
 
 Where the page is silent the oracle takes these readings (the same ones the
 CUDA path implements):
@@ -46,6 +48,11 @@ CUDA path implements):
       (row, offset_lo, offset_hi, 0), row = (b H + h) nQ + i.
   R8  attention logits z = q.k/sqrt(d) - log π_j over the valid tokens of the
       sampled blocks; softmax and value sum in fp64.
+  R9  planner variants: top-k = the s largest S_j (ties to the lower j; scores
+      ranked by the order-preserving key of their fp32 bit pattern, so +0 ranks
+      above -0 and NaN below every number), log π = 0; "no IPW" = the SIP draw
+      with log π = 0; "uniform" = the SIP fixed point and draw on a constant
+      score row (π_j = s/nK up to the 2^-32 fixed point and the trimmed tail).
 """
 
 from __future__ import annotations
@@ -320,6 +327,44 @@ def plan_row(S: np.ndarray, s: int, seed: int, offset: int, row: int):
     idx = systematic_sample(qp, order, U, s)
     logpi = np.array([math.log(int(qp[j]) / TWO32) for j in idx], dtype=np.float64)
     return idx.astype(np.int32), logpi.astype(np.float32), qp
+
+
+def score_key(S: np.ndarray) -> np.ndarray:
+    """Order-preserving uint32 key of fp32 scores (R9): larger score, larger key; NaN -> 0."""
+    b = np.asarray(S, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    neg = (b >> 31) == 1
+    key = np.where(neg, (~b) & 0xFFFFFFFF, b | 0x80000000)
+    key = np.where(np.isnan(np.asarray(S, dtype=np.float32)), 0, key)
+    return key.astype(np.uint64)
+
+
+def topk_row(S: np.ndarray, s: int):
+    """[ABL] deterministic top-k: the s largest scores, ties to the lower index (R9).
+
+    Returns (idx ascending int32 [s], logπ = 0 fp32 [s]).  A plain sort of
+    (-key, index) pairs.
+    """
+    key = score_key(S)
+    ranked = sorted(range(len(key)), key=lambda j: (-int(key[j]), j))
+    idx = np.array(sorted(ranked[:s]), dtype=np.int32)
+    return idx, np.zeros(s, dtype=np.float32)
+
+
+def plan_row_variant(S: np.ndarray, s: int, seed: int, offset: int, row: int, mode: str):
+    """One query block's plan under a planner variant (R9): "sip", "sip_no_ipw",
+    "uniform" or "topk".  Returns (idx ascending int32 [s], logπ fp32 [s])."""
+    if mode == "sip":
+        idx, lp, _ = plan_row(S, s, seed, offset, row)
+        return idx, lp
+    if mode == "sip_no_ipw":
+        idx, _, _ = plan_row(S, s, seed, offset, row)
+        return idx, np.zeros(s, dtype=np.float32)
+    if mode == "uniform":
+        idx, lp, _ = plan_row(np.ones(len(S), dtype=np.float32), s, seed, offset, row)
+        return idx, lp
+    if mode == "topk":
+        return topk_row(S, s)
+    raise ValueError(mode)
 
 
 def sample_row(pi: np.ndarray, s: int, seed: int, offset: int, row: int):

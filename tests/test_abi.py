@@ -78,5 +78,9 @@ def test_null_and_misaligned_pointers_rejected_before_any_cuda_call():
     assert L.ab_plan(P, fake, 0, 1, 0, fake, fake, null) == -1
     assert L.ab_plan(P, fake, 300, 1, 0, fake, fake, null) == -1
     assert L.ab_sample(P, fake, 32, 1, 0, null, fake, null) == -1
+    assert L.ab_plan_variant(P, fake, 32, 1, 0, 7, fake, fake, null) == -1   # unknown mode
+    assert L.ab_plan_variant(P, fake, 32, 1, 0, -1, fake, fake, null) == -1
+    assert L.ab_plan_variant(P, null, 32, 1, 0, 3, fake, fake, null) == -1   # top-k needs S
+    assert L.ab_plan_variant(P, fake, 300, 1, 0, 2, fake, fake, null) == -1  # s > nK
     assert L.ab_attn_dense(P, fake, null, fake, fake, null) == -1
     assert L.ab_attn(None, fake, fake, fake, fake, fake, 32, fake, null) == -1

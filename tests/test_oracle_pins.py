@@ -384,3 +384,61 @@ def test_philox_round_structure_against_numpy_philox4x64():
         c1 = list(ctr)
         c1[0] += 1  # no carry for these draws (< 2^63)
         assert got == list(O.philox4(c1, key, 10, **c64))
+
+
+# ---------------------------------------------------------------- planner variants (R9)
+
+def test_topk_hand_example():
+    # scores 0.1 0.3 0.3 -0 +0 NaN 0.2, s = 4: the two 0.3 (j = 1, 2), 0.2 (j = 6), 0.1 (j = 0)
+    S = np.array([0.1, 0.3, 0.3, -0.0, 0.0, np.nan, 0.2], np.float32)
+    idx, lp = O.topk_row(S, 4)
+    assert idx.tolist() == [0, 1, 2, 6] and (lp == 0).all()
+    # s = 5 reaches the zeros: +0 ranks above -0
+    assert O.topk_row(S, 5)[0].tolist() == [0, 1, 2, 4, 6]
+    # s = 7: everything, NaN last
+    assert O.topk_row(S, 7)[0].tolist() == list(range(7))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_invariants_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    nK = int(rng.integers(5, 300))
+    S = (rng.integers(0, 7, nK) / 7.0).astype(np.float32)  # many exact ties
+    s = int(rng.integers(1, nK + 1))
+    idx, _ = O.topk_row(S, s)
+    assert len(idx) == s and (np.diff(idx) > 0).all()
+    chosen = np.zeros(nK, bool)
+    chosen[idx] = True
+    if s < nK:
+        lo = S[chosen].min()
+        hi = S[~chosen].max()
+        assert lo >= hi
+        # at the boundary value every chosen index precedes every unchosen one
+        eq = np.nonzero(S == lo)[0]
+        if (S[~chosen] == lo).any():
+            assert eq[chosen[eq]].max() < eq[~chosen[eq]].min()
+
+
+def test_uniform_variant_closed_forms():
+    # nK = 8, s = 2: every q' = 2^30 exactly; the draw is the block holding U and the one
+    # holding U + 2^32, i.e. {U >> 30, (U >> 30) + 4}
+    row, seed, off = 5, 11, 2
+    idx, lp = O.plan_row_variant(np.zeros(8, np.float32), 2, seed, off, row, "uniform")
+    U = O.plan_uniform(row, seed, off)
+    assert idx.tolist() == [U >> 30, (U >> 30) + 4]
+    assert np.allclose(lp, np.log(0.25), rtol=0, atol=1e-7)
+    # nK = 3, s = 1: lambda = the smallest fp32 with 3 floor(lambda 2^32) >= 2^32; fp32 near
+    # 1/3 has spacing 2^-25, so q = ceil(2^32/3) rounded up to a multiple of 2^7, and the
+    # last block is trimmed to 2^32 - 2q
+    qp, order, _ = O.inclusion_fixed_point(np.ones(3, np.float32), 1)
+    q = -(-((1 << 32) // 3 + 1) // 128) * 128
+    assert [int(x) for x in qp] == [q, q, (1 << 32) - 2 * q]
+
+
+def test_no_ipw_variant_is_the_sip_draw_unweighted():
+    rng = np.random.default_rng(3)
+    S = rng.random(200).astype(np.float32)
+    S /= S.sum()
+    a = O.plan_row_variant(S, 20, 7, 1, 9, "sip")
+    b = O.plan_row_variant(S, 20, 7, 1, 9, "sip_no_ipw")
+    assert np.array_equal(a[0], b[0]) and (b[1] == 0).all() and (a[1] <= 0).all()
