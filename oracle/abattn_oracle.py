@@ -418,6 +418,31 @@ def dense_attention(Qr: np.ndarray, Kh: np.ndarray, Vh: np.ndarray) -> np.ndarra
     return (p @ Vh) / p.sum(1, keepdims=True)
 
 
+def block_attention_mass(Qb: np.ndarray, Kh: np.ndarray, kv_block: int) -> np.ndarray:
+    """Dense softmax mass of each KV block, averaged over the query block's rows, fp64.
+
+    m_j = (1/n) Σ_q Σ_{t in block j} softmax_t(q.k/sqrt(d)); Σ_j m_j = 1.  The quantity
+    whose top-s the selector tries to find ([IBCS] "which KV blocks matter"; the ablation
+    paragraph's attention-mass figures).  Measurement only.
+    """
+    N, d = Kh.shape
+    z = (Qb @ Kh.T) / math.sqrt(d)
+    z -= z.max(1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(1, keepdims=True)
+    nK = -(-N // kv_block)
+    padded = np.zeros((Qb.shape[0], nK * kv_block))
+    padded[:, :N] = p
+    return padded.reshape(Qb.shape[0], nK, kv_block).sum(2).mean(0)
+
+
+def mass_topk_row(mass: np.ndarray, s: int) -> np.ndarray:
+    """The s blocks of largest dense attention mass (ties to the lower index), ascending:
+    the oracle top-k the selector's choices are measured against."""
+    ranked = sorted(range(len(mass)), key=lambda j: (-float(mass[j]), j))
+    return np.array(sorted(ranked[:s]), dtype=np.int32)
+
+
 def ht_estimates(Qb, Kh, Vh, idx, qp, kv_block):
     """Horvitz–Thompson numerator [n, d] and denominator [n] of one sample, fp64.
 

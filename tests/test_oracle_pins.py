@@ -442,3 +442,31 @@ def test_no_ipw_variant_is_the_sip_draw_unweighted():
     a = O.plan_row_variant(S, 20, 7, 1, 9, "sip")
     b = O.plan_row_variant(S, 20, 7, 1, 9, "sip_no_ipw")
     assert np.array_equal(a[0], b[0]) and (b[1] == 0).all() and (a[1] <= 0).all()
+
+
+# ---------------------------------------------------------------- dense attention mass
+
+def test_block_mass_sums_to_one_and_matches_brute_force():
+    rng = np.random.default_rng(12)
+    N, d, bk = 37, 8, 4          # ragged last block of 1 token
+    Qb = rng.standard_normal((5, d))
+    Kh = rng.standard_normal((N, d))
+    m = O.block_attention_mass(Qb, Kh, bk)
+    assert m.shape == (10,) and abs(m.sum() - 1) < 1e-12
+    # brute force: per query, per token softmax, summed per block, averaged over queries
+    ref = np.zeros(10)
+    for q in Qb:
+        w = [math.exp(float(q @ k) / math.sqrt(d)) for k in Kh]
+        tot = sum(w)
+        for t, wt in enumerate(w):
+            ref[t // bk] += wt / tot / len(Qb)
+    assert np.allclose(m, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_block_mass_of_identical_keys_is_proportional_to_block_size():
+    N, d, bk = 10, 4, 4           # blocks of 4, 4, 2 identical keys
+    Kh = np.ones((N, d))
+    m = O.block_attention_mass(np.ones((3, d)), Kh, bk)
+    assert np.allclose(m, [0.4, 0.4, 0.2], rtol=0, atol=1e-15)
+    assert O.mass_topk_row(m, 1).tolist() == [0]   # tie: the lower index
+    assert O.mass_topk_row(m, 2).tolist() == [0, 1]
