@@ -276,6 +276,30 @@ def run_ours(args, world, rank, local):
     sp_bytes = select_plan_bytes(w)
     sp_gbs = sp_bytes / ((sel_ms + plan_ms) * 1e-3) / 1e9
 
+    # select + plan overlapped across head groups on two streams (ab_select_plan), timed
+    # after the step loop on the same inputs
+    sp_over_ms = None
+    if args.only == "all":
+        s2 = torch.cuda.Stream(device=dev)
+        for i in range(2):
+            ab.ab_select_plan(p, Q, K, S, ws, w.s, w.philox_seed, i, idx, lp, groups=2, stream2=s2)
+        torch.cuda.synchronize()
+        o0, o1 = E(), E()
+        o0.record(stream)
+        for i in range(3):  # two head groups: the least slow split measured (no split is faster)
+            ab.ab_select_plan(p, Q, K, S, ws, w.s, w.philox_seed, i, idx, lp, groups=2, stream2=s2)
+        o1.record(stream)
+        torch.cuda.synchronize()
+        sp_over_ms = max_over_ranks(o0.elapsed_time(o1) / 3, world)
+        st = ab.ab_get_status()
+        if st != 0:
+            raise RuntimeError(f"device status after select+plan: {ab.ab_status_string(st)}")
+    # select's exponential work at the special-function rate (16 per clock per SM)
+    sm_hz = (clk.summary().get("sm_mhz") or 1800.0) * 1e6
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sel_exp = 2 * w.clusters * w.B * w.H * w.nQ * w.nK
+    sel_sfu_ms = sel_exp / (16 * n_sms * sm_hz) * 1e3
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e and args.only == "all":
@@ -298,6 +322,11 @@ def run_ours(args, world, rank, local):
         "select_ms": round(sel_ms, 3), "plan_ms": round(plan_ms, 3),
         "select_plan_gbs": round(sp_gbs, 1),
         "select_plan_frac_of_hbm": round(sp_gbs / peaks["hbm_gbs"], 4),
+        "select_sfu_bound_ms": round(sel_sfu_ms, 3),
+        "select_sfu_frac": round(sel_sfu_ms / sel_ms, 4) if run_select else None,
+        "select_plan_overlapped_ms": None if sp_over_ms is None else round(sp_over_ms, 3),
+        "select_plan_overlapped_frac_of_hbm": (None if sp_over_ms is None else
+                                               round(sp_bytes / (sp_over_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)),
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,false>",
                      "achieved": round(attn_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak_t, 4),

@@ -18,7 +18,8 @@ import os
 
 __all__ = [
     "ABError", "ABParams", "params", "lib", "ab_workspace_bytes", "ab_select",
-    "ab_select_debug", "ab_plan", "ab_plan_variant", "ab_sample", "ab_attn", "ab_attn_dense",
+    "ab_select_debug", "ab_select_plan", "ab_plan", "ab_plan_variant", "ab_sample", "ab_attn",
+    "ab_attn_dense",
     "ab_get_status", "ab_status_string", "ab_version", "LIB_PATH", "PLAN_MODES",
 ]
 
@@ -59,6 +60,7 @@ _SIGS = {
     "ab_select_debug": [_P, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp],
     "ab_plan": [_P, _vp, _i, _u64, _u64, _vp, _vp, _vp],
     "ab_plan_variant": [_P, _vp, _i, _u64, _u64, _i, _vp, _vp, _vp],
+    "ab_select_plan": [_P, _vp, _vp, _vp, _vp, _sz, _i, _u64, _u64, _vp, _vp, _i, _vp, _vp],
     "ab_sample": [_P, _vp, _i, _u64, _u64, _vp, _vp, _vp],
     "ab_attn": [_P, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp],
     "ab_attn_dense": [_P, _vp, _vp, _vp, _vp, _vp],
@@ -148,6 +150,19 @@ def ab_plan(p, S, s, seed, offset, idx, logpi, stream=None):
     _check(lib().ab_plan(ctypes.byref(p), _ptr(S, "S", torch.float32), int(s), int(seed), int(offset),
                          _ptr(idx, "idx", torch.int32), _ptr(logpi, "logpi", torch.float32),
                          _stream(stream)), "ab_plan")
+
+
+def ab_select_plan(p, Q, K, S, ws, s, seed, offset, idx, logpi, groups=0, stream=None,
+                   stream2=None):
+    """ab_select then ab_plan, overlapped across head groups on ``stream`` and ``stream2``."""
+    import torch
+
+    _check(lib().ab_select_plan(ctypes.byref(p), _ptr(Q, "Q", torch.bfloat16),
+                                _ptr(K, "K", torch.bfloat16), _ptr(S, "S", torch.float32),
+                                _ptr(ws, "ws"), ws.numel() * ws.element_size(), int(s), int(seed),
+                                int(offset), _ptr(idx, "idx", torch.int32),
+                                _ptr(logpi, "logpi", torch.float32), int(groups), _stream(stream),
+                                None if stream2 is None else _stream(stream2)), "ab_select_plan")
 
 
 def ab_plan_variant(p, S, s, seed, offset, mode, idx, logpi, stream=None):

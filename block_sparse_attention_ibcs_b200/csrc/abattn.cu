@@ -123,8 +123,9 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
 }
 
 ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t offset,
-                   int mode, int32_t* idx, float* logpi, cudaStream_t st) {
+                   int mode, int32_t* idx, float* logpi, cudaStream_t st, long long row0 = 0) {
   PlanArgs a;
+  a.row0 = (int)row0;
   a.S = S;
   a.idx = idx;
   a.logpi = logpi;
@@ -264,6 +265,31 @@ ab_status plan_common(const ab_params* p, const float* S, int s, uint64_t seed, 
   return run_plan(d, S, s, seed, offset, mode, idx, logpi, (cudaStream_t)stream);
 }
 
+// Select then plan for heads [bh0, bh0 + n) of the flattened (b, h) order: the slice is a
+// problem with B*H = n on offset pointers (every kernel of both stages works per (b, h)).
+ab_status select_plan_slice(const Dims& d, long long bh0, long long n, const void* Q,
+                            const void* K, float* S, void* ws, int s, uint64_t seed,
+                            uint64_t offset, int32_t* idx, float* logpi, cudaStream_t st_sel,
+                            cudaStream_t st_plan, cudaEvent_t ev) {
+  Dims g = d;
+  g.BH = n;
+  const size_t qk = (size_t)bh0 * d.N * d.d;  // elements
+  const void* Qg = (const uint16_t*)Q + qk;
+  const void* Kg = (const uint16_t*)K + qk;
+  float* Sg = S + (size_t)bh0 * d.nQ * d.nK;
+  Workspace wsp = carve(g, ws);
+  ab_status r = (d.d == 128) ? run_select<128>(g, Qg, Kg, Sg, wsp, nullptr, st_sel)
+                             : run_select<64>(g, Qg, Kg, Sg, wsp, nullptr, st_sel);
+  if (r != AB_OK) return r;
+  if (st_plan != st_sel) {
+    if (cudaEventRecord(ev, st_sel) != cudaSuccess || cudaStreamWaitEvent(st_plan, ev, 0) != cudaSuccess)
+      return launch_status();
+  }
+  const size_t rows = (size_t)bh0 * d.nQ;
+  return run_plan(g, Sg, s, seed, offset, AB_PLAN_SIP, idx + rows * s, logpi + rows * s, st_plan,
+                  (long long)rows);
+}
+
 }  // namespace
 
 extern "C" {
@@ -291,6 +317,44 @@ ab_status ab_select_debug(const ab_params* p, const void* Q, const void* K, floa
 ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,
                   int32_t* idx, float* logpi, void* stream) {
   return plan_common(p, S, s, seed, offset, AB_PLAN_SIP, idx, logpi, stream);
+}
+
+ab_status ab_select_plan(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
+                         size_t ws_bytes, int s, uint64_t seed, uint64_t offset, int32_t* idx,
+                         float* logpi, int groups, void* stream, void* stream2) {
+  Dims d;
+  ab_status r = check_params(p, &d);
+  if (r != AB_OK) return r;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(S)) return AB_ERR_INVALID_ARG;
+  if (!idx || !logpi || ((uintptr_t)idx & 3) || ((uintptr_t)logpi & 3)) return AB_ERR_INVALID_ARG;
+  if (s < 1 || s > d.nK) return AB_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255)) return AB_ERR_WORKSPACE;
+  if (ws_bytes < carve(d, ws).bytes) return AB_ERR_WORKSPACE;
+  cudaStream_t sa = (cudaStream_t)stream, sb = (cudaStream_t)stream2;
+  if (!sb || sb == sa) return select_plan_slice(d, 0, d.BH, Q, K, S, ws, s, seed, offset, idx, logpi, sa, sa, nullptr);
+  // automatic: no split.  On B200 at the Wan2.1-14B shape every split measured slower than
+  // the two stages back to back (2 groups: 7.06 vs 6.89 ms; 8: 9.1 ms): both stages are
+  // compute-bound and their CTAs do not fit on one SM together (shared memory).
+  long long G = groups > 0 ? groups : 1;
+  if (G > d.BH) G = d.BH;
+  // events: one per group (select of group g done -> plan of group g may start), one for the end
+  cudaEvent_t evs[65];
+  if (G > 64) G = 64;
+  for (long long g = 0; g <= G; ++g)
+    if (cudaEventCreateWithFlags(&evs[g], cudaEventDisableTiming) != cudaSuccess) {
+      for (long long k = 0; k < g; ++k) cudaEventDestroy(evs[k]);
+      return launch_status();
+    }
+  r = AB_OK;
+  for (long long g = 0; g < G && r == AB_OK; ++g) {
+    const long long b0 = d.BH * g / G, b1 = d.BH * (g + 1) / G;
+    r = select_plan_slice(d, b0, b1 - b0, Q, K, S, ws, s, seed, offset, idx, logpi, sa, sb, evs[g]);
+  }
+  // the caller's stream sees every plan as done
+  if (r == AB_OK && (cudaEventRecord(evs[G], sb) != cudaSuccess || cudaStreamWaitEvent(sa, evs[G], 0) != cudaSuccess))
+    r = launch_status();
+  for (long long g = 0; g <= G; ++g) cudaEventDestroy(evs[g]);  // released once their work is done
+  return r;
 }
 
 ab_status ab_plan_variant(const ab_params* p, const float* S, int s, uint64_t seed, uint64_t offset,

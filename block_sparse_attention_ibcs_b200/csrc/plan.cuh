@@ -42,6 +42,9 @@ struct PlanArgs {
   int nK, s;
   uint64_t seed, offset;
   int mode;         // ab_plan_mode: SIP, SIP without inverse-probability weights, uniform
+  int row0;         // row index of this launch's first row in the whole (b, h, i) order
+                    // (the Philox counter uses it: a launch over a slice of heads draws as
+                    // the full launch would)
 };
 
 // Philox4x32-10 (Salmon et al., SC'11), word 0 of the output block.
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   uint64_t sat_before, rest_before, n_sat, tot_rest;
   block_exscan2_u64(my_sat, my_rest, red, red2, sat_before, rest_before, n_sat, tot_rest);
 
-  const uint32_t U = philox4x32_10_w0((uint32_t)row, (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
+  const uint32_t U = philox4x32_10_w0((uint32_t)(a.row0 + row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
                                       0u, (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
   // lattice points U + k 2^32 below x, for 0 <= x <= s 2^32 (U < 2^32)
   const uint64_t CB = TWO32 - 1u - (uint64_t)U;

@@ -114,6 +114,21 @@ ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint
 ab_status ab_sample(const ab_params* p, const float* pi, int s, uint64_t seed,
                     uint64_t offset, int32_t* idx, float* logpi, void* stream);
 
+/* ab_select followed by ab_plan (SIP), with the two stages overlapped across heads: the
+ * B*H heads are cut into `groups` slices (0 = automatic: 1, i.e. no split, which measured
+ * fastest on B200 at the Wan2.1-14B shape; at most 64 and at most B*H);
+ * slice g is scored on `stream` and then planned on `stream2` while slice g+1 is scored,
+ * so the planner's integer work overlaps the selector's tensor-core and exponential work.
+ * Results are bit-identical to ab_select then ab_plan with the same arguments (the
+ * planner's Philox counter uses each row's index in the whole tensor).  On return, work
+ * enqueued later on `stream` runs after both stages; `stream2` must differ from `stream`
+ * to overlap (NULL or equal: the two stages run one after the other on `stream`).  The
+ * workspace is the one ab_select needs for the whole problem.  Arguments otherwise as
+ * ab_select and ab_plan.                                                               */
+ab_status ab_select_plan(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
+                         size_t ws_bytes, int s, uint64_t seed, uint64_t offset, int32_t* idx,
+                         float* logpi, int groups, void* stream, void* stream2);
+
 /* Planner variants for the ablations on the AB-Attention page (the selection rules SIP
  * is compared against).  Same arguments and output layout as ab_plan, plus `mode`:
  *   AB_PLAN_SIP         exactly ab_plan.

@@ -78,6 +78,12 @@ def test_null_and_misaligned_pointers_rejected_before_any_cuda_call():
     assert L.ab_plan(P, fake, 0, 1, 0, fake, fake, null) == -1
     assert L.ab_plan(P, fake, 300, 1, 0, fake, fake, null) == -1
     assert L.ab_sample(P, fake, 32, 1, 0, null, fake, null) == -1
+    assert L.ab_select_plan(P, fake, fake, fake, fake, 1 << 30, 0, 1, 0, fake, fake, 0, null,
+                            null) == -1                                     # s < 1
+    assert L.ab_select_plan(P, fake, fake, fake, null, 1 << 30, 32, 1, 0, fake, fake, 0, null,
+                            null) == -5                                     # no workspace
+    assert L.ab_select_plan(P, fake, fake, fake, fake, 16, 32, 1, 0, fake, fake, 0, null,
+                            null) == -5                                     # workspace too small
     assert L.ab_plan_variant(P, fake, 32, 1, 0, 7, fake, fake, null) == -1   # unknown mode
     assert L.ab_plan_variant(P, fake, 32, 1, 0, -1, fake, fake, null) == -1
     assert L.ab_plan_variant(P, null, 32, 1, 0, 3, fake, fake, null) == -1   # top-k needs S
