@@ -362,18 +362,49 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
     h2d = (hostQ.numel() + hostK.numel() + 3 * reuse * hostQ.numel()) * 2
     d2h = reuse * hostQ.numel() * 2
 
-    def step(i):
-        dQ.copy_(hostQ, non_blocking=True)
-        dK.copy_(hostK, non_blocking=True)
-        ab.ab_select(p, dQ, dK, S, ws)
-        ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp)
-        for c in range(reuse):
-            for dst, src in zip(dP[c], hostP[c]):
-                dst.copy_(src, non_blocking=True)
-            ab.ab_attn(p, dP[c][0], dP[c][1], dP[c][2], idx, lp, w.s, dO[c])
-            hostO[c].copy_(dO[c], non_blocking=True)
-
+    # Three streams: host->device copies (cs), compute (the current stream), device->host
+    # copies (ds).  The copy of attention call c's inputs overlaps the calls before it, and
+    # each output's copy back overlaps the calls after it; events keep every buffer from
+    # being overwritten before its previous reader is done.
     stream = torch.cuda.current_stream()
+    cs = torch.cuda.Stream(device=dev)
+    ds = torch.cuda.Stream(device=dev)
+    prev = {"sel": None, "attn": [None] * reuse, "d2h": [None] * reuse}
+
+    def ev_on(st):
+        e = torch.cuda.Event()
+        e.record(st)
+        return e
+
+    def step(i):
+        with torch.cuda.stream(cs):
+            if prev["sel"] is not None:
+                cs.wait_event(prev["sel"])
+            dQ.copy_(hostQ, non_blocking=True)
+            dK.copy_(hostK, non_blocking=True)
+            qk_ready = ev_on(cs)
+            ready = []
+            for c in range(reuse):
+                if prev["attn"][c] is not None:
+                    cs.wait_event(prev["attn"][c])
+                for dst, src in zip(dP[c], hostP[c]):
+                    dst.copy_(src, non_blocking=True)
+                ready.append(ev_on(cs))
+        stream.wait_event(qk_ready)
+        ab.ab_select(p, dQ, dK, S, ws, stream)
+        prev["sel"] = ev_on(stream)
+        ab.ab_plan(p, S, w.s, w.philox_seed, i, idx, lp, stream)
+        for c in range(reuse):
+            stream.wait_event(ready[c])
+            if prev["d2h"][c] is not None:
+                stream.wait_event(prev["d2h"][c])
+            ab.ab_attn(p, dP[c][0], dP[c][1], dP[c][2], idx, lp, w.s, dO[c], stream)
+            prev["attn"][c] = ev_on(stream)
+            with torch.cuda.stream(ds):
+                ds.wait_event(prev["attn"][c])
+                hostO[c].copy_(dO[c], non_blocking=True)
+                prev["d2h"][c] = ev_on(ds)
+
     for i in range(2):
         step(i)
     steps = max(1, min(args.steps, 3))
@@ -381,8 +412,12 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    cs.wait_stream(stream)  # nothing of the timed steps starts before t0
+    ds.wait_stream(stream)
     for i in range(steps):
         step(100 + i)
+    stream.wait_stream(cs)  # ... and t1 follows every copy of them
+    stream.wait_stream(ds)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
