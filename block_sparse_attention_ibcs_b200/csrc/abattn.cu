@@ -147,7 +147,7 @@ ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t
     }
     return launch_status();
   }
-  if (d.nK <= PLAN_SMEM_MAX_FLOATS) {
+  if (d.nK <= PLAN_STAGE_MAX_FLOATS) {
     const size_t smem = (size_t)((d.nK + 3) / 4) * 16;  // row padded to whole float4s
     // per-device attribute; cheap enough to set on every launch
     if (cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -17,13 +17,13 @@
 //
 // One CTA of PLAN_THREADS threads per row.  The row is staged in shared memory when it
 // fits, otherwise re-read from global memory (L2) on each pass.  Passes over the row:
-// staging with the positive count and sum; a water-filling estimate of lambda (usually
-// one pass); F at the estimate and at one Newton step from it (these bracket lambda* to
-// one ulp on typical rows; otherwise a doubling search and bisection follow); the codes
-// (q_j or "saturated") with per-thread sums; and the output pass.  The number selected
-// in each thread's contiguous chunk needs no pass of its own: non-saturated intervals are
-// shorter than 2^32, so the chunk's blocks hold exactly the lattice points of the chunk's
-// (contiguous) interval.
+// staging with the positive count and sum; F at lambda0 = s / sum(S) (with the sum of the
+// unsaturated scores) and at one Newton step from it -- these bracket lambda* to one ulp
+// on typical rows, otherwise a doubling search and bisection follow; and the output pass.
+// After staging every pass walks the thread's contiguous chunk, so F(lambda*) already gives
+// each thread its saturated count and q sum; the number drawn in a chunk needs no pass:
+// non-saturated intervals are shorter than 2^32, so the chunk's blocks hold exactly the
+// lattice points of the chunk's (contiguous) interval.
 #pragma once
 
 #include "common.cuh"
@@ -32,7 +32,12 @@ namespace abattn {
 
 constexpr int PLAN_THREADS = 512;
 constexpr int PLAN_WARPS = PLAN_THREADS / 32;
-constexpr int PLAN_SMEM_MAX_FLOATS = 40 * 1024;  // 160 KB of staged row
+constexpr int PLAN_SMEM_MAX_FLOATS = 40 * 1024;  // 160 KB of staged row (top-k keys)
+// The SIP planner stages a row only while two CTAs still fit on an SM (112 KB each):
+// measured on B200, one staged CTA per SM (e.g. 29,700 blocks) is slower than re-reading
+// the row from L2 with two CTAs per SM (4.9 vs 4.0 ms at the HunyuanVideo shape), while at
+// 18,900 blocks staging wins (2.7 vs 3.6 ms).
+constexpr int PLAN_STAGE_MAX_FLOATS = 28 * 1024;
 constexpr uint64_t TWO32 = 1ull << 32;
 
 struct PlanArgs {
@@ -166,17 +171,33 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   const int tid = threadIdx.x;
   const int nK = a.nK;
   const float* grow = a.S + (size_t)row * nK;
-  const float* srow = grow;
   const bool uniform = a.mode == AB_PLAN_UNIFORM;
-  // score j of the row when it is not staged (the uniform variant reads no scores)
-  auto sv_at = [&](int j) -> float { return uniform ? 1.f : __ldg(grow + j); };
-  const int nK4 = (nK + 3) >> 2;  // staged row padded with zeros to whole float4s
+  const int nK4 = (nK + 3) >> 2;  // the row in whole float4s (zeros past nK)
   const uint64_t s = (uint64_t)a.s;
   const uint64_t target = s * TWO32;
+  // This thread's contiguous chunk of float4s (an odd count keeps eight consecutive
+  // threads' 16-byte shared loads on distinct banks); every pass after staging walks it.
+  const int per4 = ((nK4 + PLAN_THREADS - 1) / PLAN_THREADS) | 1;
+  const int c0 = min(nK4, tid * per4), c1 = min(nK4, c0 + per4);
+  auto load4 = [&](int i) -> float4 {
+    if (STAGED) return reinterpret_cast<const float4*>(srow_smem)[i];
+    float4 v;
+    const int j = 4 * i;
+    if (uniform) {
+      v = make_float4(j < nK ? 1.f : 0.f, j + 1 < nK ? 1.f : 0.f, j + 2 < nK ? 1.f : 0.f,
+                      j + 3 < nK ? 1.f : 0.f);
+    } else {
+      v.x = (j < nK) ? __ldg(grow + j) : 0.f;
+      v.y = (j + 1 < nK) ? __ldg(grow + j + 1) : 0.f;
+      v.z = (j + 2 < nK) ? __ldg(grow + j + 2) : 0.f;
+      v.w = (j + 3 < nK) ? __ldg(grow + j + 3) : 0.f;
+    }
+    return v;
+  };
 
   // ---- positive blocks and their total score (fewer than s positive blocks = budget
   // unreachable); per-thread sums in compensated fp32, block sum in fp64.  With the row
-  // staged in shared memory this pass also copies it there.
+  // staged in shared memory this pass also copies it there (coalesced, strided).
   uint64_t npos = 0;
   double tot = 0.0;
   {
@@ -213,9 +234,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         acc(v.z);
         acc(v.w);
       }
-      srow = srow_smem;  // read only after the barriers of the block sum below
+      // read by other threads only after the barriers of the block sum below
     } else {
-      for (int j = tid; j < nK; j += PLAN_THREADS) acc(sv_at(j));
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        acc(v.x);
+        acc(v.y);
+        acc(v.z);
+        acc(v.w);
+      }
     }
     tot = (double)sum - (double)comp;
   }
@@ -225,84 +252,96 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   // ---- lambda*: the smallest positive fp32 (bit pattern in (0, 0x7F800000]) with
   // F(lambda) >= s 2^32.  F is monotone in the bit pattern, so any search that brackets
   // the boundary and bisects finds the same lambda as a full 31-step bisection.
-  auto F = [&](uint32_t bits) -> uint64_t {
+  // F(bits) also leaves this thread's part -- its saturated count and the sum of its other
+  // q_j -- in (ev_nsat, ev_q), and with `want_rest` the block sum of the unsaturated scores.
+  uint32_t ev_nsat = 0;
+  uint64_t ev_q = 0;
+  auto F = [&](uint32_t bits, bool want_rest, double* rest_out) -> uint64_t {
     const float lam = __uint_as_float(bits);
-    uint64_t part = 0;
-    if (STAGED) {
-      const float4* s4 = reinterpret_cast<const float4*>(srow);
-      for (int j = tid; j < nK4; j += PLAN_THREADS) {
-        const float4 v = s4[j];
-        add_q(lam, v.x, part);
-        add_q(lam, v.y, part);
-        add_q(lam, v.z, part);
-        add_q(lam, v.w, part);
+    uint32_t ns = 0;
+    uint64_t qs = 0;
+    float rest = 0.f;
+    for (int i = c0; i < c1; ++i) {
+      const float4 v = load4(i);
+      const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t q;
+        const bool sat = fixed_q32(lam, x4[k], q);
+        ns += sat;
+        qs += sat ? 0u : q;
+        if (want_rest && !sat && x4[k] > 0.f) rest += x4[k];
       }
-    } else {
-      for (int j = tid; j < nK; j += PLAN_THREADS) add_q(lam, sv_at(j), part);
+    }
+    ev_nsat = ns;
+    ev_q = qs;
+    uint64_t part = ((uint64_t)ns << 32) + qs;  // per thread below 2^39
+    if (want_rest) {
+      double r = rest;
+      block_sum_cd(part, r, red, redd);
+      *rest_out = r;
+      return part;
     }
     return block_sum_u64(part, red);
   };
   uint32_t lo = 0u, hi = 0x7F800000u;
+  bool hi_known = false;  // whether (hi_nsat, hi_q) hold this thread's part of F(hi)
+  uint32_t hi_nsat = 0;
+  uint64_t hi_q = 0;
+  auto take_hi = [&](uint32_t bits) {
+    hi = bits;
+    hi_nsat = ev_nsat;
+    hi_q = ev_q;
+    hi_known = true;
+  };
   if (reachable) {
-    // Water filling in fp64 (a starting point only): lambda <- (s - |saturated|) / (sum of
-    // the unsaturated scores) until the saturated set stops growing; in practice one or
-    // two rounds, ending within an ulp or two of lambda*.
-    double lam_w = (tot > 0.0) ? (double)a.s / tot : 0.0;
-    double rest_est = tot;
-    for (int it = 0; it < 32 && lam_w > 0.0; ++it) {
-      uint64_t nsat = 0;
-      double rest = 0.0;
-      const float lw = (float)lam_w;
-      {
-        float sum = 0.f, comp = 0.f;
-        for (int j = tid; j < nK; j += PLAN_THREADS) {
-          const float sv = STAGED ? srow[j] : sv_at(j);
-          if (sv > 0.f) {
-            if (__fmul_rn(lw, sv) >= 1.f) {
-              ++nsat;
-            } else {
-              const float y = sv - comp, t2 = sum + y;
-              comp = (t2 - sum) - y;
-              sum = t2;
-            }
-          }
-        }
-        rest = (double)sum - (double)comp;
-      }
-      block_sum_cd(nsat, rest, red, redd);
-      rest_est = rest;
-      if (nsat >= (uint64_t)a.s || !(rest > 0.0)) break;
-      const double nxt = (double)((uint64_t)a.s - nsat) / rest;
-      if (!(nxt > lam_w)) break;  // converged (the iteration only increases)
-      lam_w = nxt;
-    }
-    const float lam_est = (float)lam_w;
-    uint32_t b = __float_as_uint(lam_est);
-    if (!(lam_est > 0.f) || !isfinite(lam_est)) b = 0x3F800000u;  // 1.0: any start works
-    uint64_t fb = F(b);
-    // one Newton step on the fixed-point sum: F grows by about rest * 2^32 per unit lambda
-    if (rest_est > 0.0 && isfinite(lam_est) && lam_est > 0.f) {
+    // Start at lambda0 = s / sum(S) and take one Newton step on the exact integer sum:
+    // F grows by about (sum of the unsaturated scores) * 2^32 per unit lambda, so the step
+    // is the water-filling update lambda <- (s - |saturated|) / (unsaturated sum).  On
+    // typical rows the two points bracket lambda* to one ulp.
+    const float lam0 = (tot > 0.0) ? (float)((double)a.s / tot) : 0.f;
+    uint32_t b = __float_as_uint(lam0);
+    if (!(lam0 > 0.f) || !isfinite(lam0)) b = 0x3F800000u;  // 1.0: any start works
+    double rest = 0.0;
+    uint64_t fb = F(b, true, &rest);
+    uint32_t b_nsat = ev_nsat;
+    uint64_t b_q = ev_q;
+    auto point_b_is_hi = [&]() {
+      hi = b;
+      hi_nsat = b_nsat;
+      hi_q = b_q;
+      hi_known = true;
+    };
+    if (rest > 0.0) {
       const double lam_n = (double)__uint_as_float(b) +
-                           ((double)target - (double)fb) / (rest_est * 4294967296.0);
+                           ((double)target - (double)fb) / (rest * 4294967296.0);
       const float lf = (float)lam_n;
       if (lf > 0.f && isfinite(lf) && __float_as_uint(lf) != b) {
         const uint32_t b2 = __float_as_uint(lf);
-        const uint64_t f2 = F(b2);
-        // keep whichever point is on the same side as the boundary search needs
-        if ((f2 >= target) == (fb >= target)) { b = b2; fb = f2; }
-        else if (b2 > b) { lo = b; hi = b2; }
-        else { lo = b2; hi = b; }
+        const uint64_t f2 = F(b2, false, nullptr);
+        if ((f2 >= target) == (fb >= target)) {  // same side: continue from the Newton point
+          b = b2;
+          fb = f2;
+          b_nsat = ev_nsat;
+          b_q = ev_q;
+        } else if (b2 > b) {
+          lo = b;
+          take_hi(b2);
+        } else {
+          lo = b2;
+          point_b_is_hi();
+        }
       }
     }
     const bool bracketed = !(lo == 0u && hi == 0x7F800000u);  // by the Newton point
     if (!bracketed) {
       if (fb >= target) {  // boundary at or below b: step down
-        hi = b;
+        point_b_is_hi();
         uint32_t step = 1;
         while (true) {
           const uint32_t cand = (hi > step) ? hi - step : 0u;
-          if (cand == 0u || F(cand) < target) { lo = cand; break; }
-          hi = cand;
+          if (cand == 0u || F(cand, false, nullptr) < target) { lo = cand; break; }
+          take_hi(cand);
           step <<= 1;
         }
       } else {  // boundary above b: step up
@@ -310,7 +349,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         uint32_t step = 1;
         while (true) {
           const uint32_t cand = (0x7F800000u - lo > step) ? lo + step : 0x7F800000u;
-          if (cand == 0x7F800000u || F(cand) >= target) { hi = cand; break; }
+          if (cand == 0x7F800000u) { hi = cand; hi_known = false; break; }
+          if (F(cand, false, nullptr) >= target) { take_hi(cand); break; }
           lo = cand;
           step <<= 1;
         }
@@ -318,34 +358,34 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     }
     while (hi - lo > 1u) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (F(mid) >= target) hi = mid; else lo = mid;
+      if (F(mid, false, nullptr) >= target) take_hi(mid); else lo = mid;
+    }
+    if (!hi_known) {  // lambda* = +inf was never evaluated (pathological rows)
+      F(hi, false, nullptr);
+      take_hi(hi);
     }
   }
   const float lam = __uint_as_float(hi);
 
-  // ---- per element code on this thread's contiguous chunk: the fixed-point q_j (< 2^32 - 255)
-  // or SAT for an inclusion probability of exactly 1 (when the budget is unreachable: every
-  // positive block is SAT and the others have code 0).  With the row staged in shared
-  // memory the codes overwrite the thread's own slots: every read of the scores by the
-  // other threads happened before the barriers of the last block sum.
-  constexpr uint32_t SAT = 0xFFFFFFFFu;
-  uint32_t* code_smem = reinterpret_cast<uint32_t*>(srow_smem);
-  auto code_from_score = [&](float sv) -> uint32_t {
-    if (reachable) {
-      uint32_t q;
-      return fixed_q32(lam, sv, q) ? SAT : q;
+  // ---- this thread's chunk: saturated count and the sum of its other q_j (budget
+  // reachable: the part of F(lambda*) kept above), or (budget unreachable) its positive
+  // blocks (pi = 1) and its other blocks (the first s - |positive| of them complete the draw)
+  uint64_t my_sat, my_rest;
+  if (reachable) {
+    my_sat = hi_nsat;
+    my_rest = hi_q;
+  } else {
+    my_sat = 0;
+    my_rest = 0;
+    for (int i = c0; i < c1; ++i) {
+      const float4 v = load4(i);
+      const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (4 * i + k >= nK) break;
+        if (x4[k] > 0.f) ++my_sat; else ++my_rest;
+      }
     }
-    return (sv > 0.f) ? SAT : 0u;
-  };
-  const int per = (nK + PLAN_THREADS - 1) / PLAN_THREADS;
-  const int j0 = min(nK, tid * per), j1 = min(nK, j0 + per);
-  // my_rest: the chunk's total q (budget reachable) or its number of code-0 blocks
-  uint64_t my_sat = 0, my_rest = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t c = code_from_score(STAGED ? srow[j] : sv_at(j));
-    if (STAGED) code_smem[j] = c;
-    if (c == SAT) ++my_sat;
-    else my_rest += reachable ? c : 1u;
   }
   uint64_t sat_before, rest_before, n_sat, tot_rest;
   block_exscan2_u64(my_sat, my_rest, red, red2, sat_before, rest_before, n_sat, tot_rest);
@@ -358,7 +398,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   // Saturated blocks come first in the layout, block k of them covering [k 2^32, (k+1) 2^32):
   // each holds exactly one lattice point, so every saturated block is drawn.  The other
   // blocks follow in ascending order; this thread's chunk covers [start, start + my_rest).
-  // With the budget unreachable, the first s - n_sat code-0 blocks (in order) complete it.
+  // With the budget unreachable, the first s - n_sat zero blocks (in order) complete it.
   const uint64_t start = n_sat * TWO32 + rest_before;
   const uint64_t need = s - min(n_sat, s);
   const uint64_t my_sel =
@@ -370,30 +410,49 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
 
   // ---- write ascending idx and the fixed-point probability (its log follows below)
   {
+    // Below the cap s 2^32, a non-saturated block [pos, pos + q) holds a lattice point iff
+    // dist < q, with dist = (U - pos) mod 2^32 the distance to the next point, and the next
+    // block starts at distance (dist - q) mod 2^32: 32-bit arithmetic.  The chunk that
+    // reaches the cap clips its intervals at s 2^32 (64-bit positions).
+    const bool capped = reachable && start + my_rest > target;
+    uint32_t dist = U - (uint32_t)start;
     uint64_t pos = start, zero_i = rest_before;
     uint64_t o = out_before;
     int32_t* oidx = a.idx + (size_t)row * a.s;
     uint32_t* oraw = reinterpret_cast<uint32_t*>(a.logpi + (size_t)row * a.s);
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t c = STAGED ? code_smem[j] : code_from_score(sv_at(j));
-      bool sel;
-      uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
-      if (c == SAT) {
-        sel = true;
-      } else if (reachable) {
-        const uint64_t st = min(pos, target), en = min(pos + c, target);
-        sel = below(en) != below(st);
-        qq = (uint32_t)(en - st);
-        pos += c;
-      } else {
-        sel = zero_i++ < need;
-      }
-      if (sel) {
-        if (o < s) {
-          oidx[o] = j;
-          oraw[o] = qq;
+    for (int i = c0; i < c1; ++i) {
+      const float4 v = load4(i);
+      const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = 4 * i + k;
+        if (j >= nK) break;
+        bool sel;
+        uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
+        if (reachable) {
+          uint32_t q;
+          if (fixed_q32(lam, x4[k], q)) {
+            sel = true;
+          } else if (!capped) {
+            sel = dist < q;
+            qq = q;
+            dist -= q;
+          } else {
+            const uint64_t st = min(pos, target), en = min(pos + q, target);
+            sel = below(en) != below(st);
+            qq = (uint32_t)(en - st);
+            pos += q;
+          }
+        } else {
+          sel = (x4[k] > 0.f) || (zero_i++ < need);
         }
-        ++o;
+        if (sel) {
+          if (o < s) {
+            oidx[o] = j;
+            oraw[o] = qq;
+          }
+          ++o;
+        }
       }
     }
   }
