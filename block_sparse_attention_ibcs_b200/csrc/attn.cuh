@@ -456,11 +456,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {  // 32 keys -> 16 TMEM columns of packed bf16 pairs
-        uint32_t pk[16];
+      for (int g = 0; g < 2; ++g) {  // 64 keys -> 32 TMEM columns of packed bf16 pairs
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * g + 2 * e;
+        for (int e = 0; e < 32; ++e) {
+          const int c0 = 64 * g + 2 * e;
           const float x0 = fmaf(z[c0], c, nmref);
           const float x1 = fmaf(z[c0 + 1], c, nmref);
           const float p0 = fast_exp2(x0);
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           ls[(2 * e + 1) & 7] += p1;
           pk[e] = pack_bf16x2_rn(p0, p1);
         }
-        tmem_st_32x32b_x16(padr + 16 * g, pk);
+        tmem_st_32x32b_x32(padr + 32 * g, pk);
       }
       const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       l_run = l_run * alpha + lsum;
