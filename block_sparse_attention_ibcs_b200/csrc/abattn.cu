@@ -71,8 +71,8 @@ Workspace carve(const Dims& d, void* base) {
   off = align256(off + (size_t)d.BH * d.nQ * CMAX * d.d * 2);
   ws.w = (float*)(b + off);
   off = align256(off + (size_t)d.BH * d.nQ * CMAX * 4);
-  ws.stats = (float*)(b + off);
-  off = align256(off + (size_t)d.BH * d.nQ * CMAX * 2 * 4);
+  ws.stats = (float*)(b + off);  // per centroid row of each 32-query-block group: key-chunk slots
+  off = align256(off + (size_t)d.BH * ((d.nQ + SC_QB - 1) / SC_QB) * SC_ROWS * SC_MAX_CHUNKS * 2 * 4);
   ws.bytes = off;
   return ws;
 }
@@ -110,15 +110,15 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
   const int pool_blocks = (int)((units + 255) / 256 < 148 * 32 ? (units + 255) / 256 : 148 * 32);
   pool_kernel<D><<<pool_blocks, 256, 0, st>>>(a);
   kmeans_kernel<D><<<(unsigned)(d.BH * d.nQ), KM_THREADS, 0, st>>>(a);
-  const unsigned sc_grid = (unsigned)(d.BH * ((d.nQ + 15) / 16));
+  const ScoreSplit sp = score_split(d.BH, d.nQ, d.nK);
   using SL = ScoreSmem<D>;
-  if (cudaFuncSetAttribute(score_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(score_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SL::ALLOC) != cudaSuccess ||
-      cudaFuncSetAttribute(score_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(score_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SL::ALLOC) != cudaSuccess)
     return launch_status();
-  score_tc_kernel<D, 1><<<sc_grid, SCT_THREADS, SL::ALLOC, st>>>(a, kDefaultTimeoutNs);
-  score_tc_kernel<D, 2><<<sc_grid, SCT_THREADS, SL::ALLOC, st>>>(a, kDefaultTimeoutNs);
+  score_kernel<D, 1><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, kDefaultTimeoutNs);
+  score_kernel<D, 2><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, kDefaultTimeoutNs);
   return launch_status();
 }
 

@@ -14,8 +14,8 @@
 //
 //   pool_kernel      Kp[bh, j, :]  = bf16(mean of block j's valid keys)
 //   kmeans_kernel    per (bh, query block): centroids (bf16) and shares (fp32)
-//   score_tc_kernel<1>  per centroid row: running max m and sum Z of exp2(logit - m)
-//   score_tc_kernel<2>  S[bh, i, j] = sum_c (w_c / Z_c) exp2(logit_cj - m_c)
+//   score_kernel<1>  per centroid row and key chunk: reference m and sum z of exp2(logit - m)
+//   score_kernel<2>  S[bh, i, j] = sum_c (w_c / Z_c) exp2(logit_cj - m_c)
 #pragma once
 
 #include "common.cuh"
@@ -31,7 +31,8 @@ struct SelectArgs {
   uint16_t* Kp;      // [BH, nK, D]
   uint16_t* cent;    // [BH, nQ, CMAX, D]
   float* w;          // [BH, nQ, CMAX]
-  float* stats;      // [BH, nQ, CMAX, 2]  (m in log2 units, Z)
+  float* stats;      // [BH, groups of 32 query blocks, 256 rows, 8 key chunks] of (m, z):
+                     // reference m (log2 units) and sum z of exp2(logit - m) per chunk
   float* S;          // [BH, nQ, nK]
   int8_t* labels;    // optional [BH, nQ*128]
   int BH, N, nQ, nK, bk, C, iters;
@@ -273,40 +274,119 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
 // ------------------------------------------------------------------ block scores (tcgen05)
 //
 // The page's batched scoring ("premises & limits": query/KV blocks scored as batched
-// matrix operations) as two tensor-core streaming passes per CTA of 16 query blocks
-// (128 centroid rows), over all pooled keys of the head in tiles of 128:
-//   PASS 1: D[centroid row, key] = C Kp^T  (A = centroids, B = key tile, both K-major).
-//           Thread r (= TMEM lane r) keeps the running max m and sum Z of exp2(logit - m).
-//   PASS 2: D[key, centroid col] = Kp C^T (A = key tile, B = centroids), so thread j owns
-//           one KV block and sums (w_c / Z_c) exp2(logit - m_c) over the 8 columns of each
-//           query block in registers; S rows are stored coalesced.
-// Roles as in the attention kernel: warps 0-3 consume TMEM, warps 4-7 stream tiles with
-// cp.async (2 stages), warp 8 allocates TMEM and issues the MMAs.
+// matrix operations) as two persistent tensor-core streaming passes.  A group is 32 query
+// blocks of one head (256 centroid rows); its key axis is cut into chunks of whole
+// 128-key tiles.  The (group, chunk) units are dealt out in order, in equal contiguous
+// runs, to one CTA per SM; a CTA walks its run as segments (consecutive units of one
+// group), loading the group's centroids once per segment.
+//   PASS 1: D[centroid row, key] = C Kp^T for the two 128-row halves of the centroids
+//           (A = centroids, B = key tile, both K-major, N = 128).  Each thread keeps a
+//           running reference m and sum z of exp2(logit - m) for one centroid row over
+//           64 of the tile's keys.  m is raised lazily: a 32-key chunk whose sum stays
+//           below 2^20 is accepted as it is (a term can then exceed 1 by at most 2^20,
+//           far from fp32 overflow); otherwise the chunk's maximum is taken and z rescaled.
+//           At the end of each key chunk the two key halves of a row are merged and the
+//           chunk's (m, z) is stored in its own slot; pass 2 merges a row's slots in chunk
+//           order, so S does not depend on how the units were dealt out to CTAs.
+//   PASS 2: D[key, centroid column] = Kp C^T (A = key tile, B = all 256 centroid rows,
+//           N = 256), so thread j owns one KV block and sums exp2(logit - m'_c) over the
+//           8 columns of each of its 8 query blocks in registers, where the share and
+//           the softmax normaliser are folded into one constant per column:
+//           w_c exp2(l - m_c) / Z_c = exp2(l - (m_c + log2 Z_c - log2 w_c)).
+//           S rows are stored coalesced.
+// Roles: warps 0-15 consume TMEM (lane quadrant = warp % 4), warps 16-17 stream tiles with
+// cp.async (3 stages), warp 18 allocates 512 TMEM columns and issues the MMAs.
 
-constexpr int SCT_THREADS = 288;
+constexpr int SC_QB = 32;                  // query blocks per group
+constexpr int SC_ROWS = SC_QB * CMAX;      // 256 centroid rows per group
+constexpr int SC_CONSUMERS = 512;          // warps 0-15
+constexpr int SC_PRODUCERS = 64;           // warps 16-17
+constexpr int SC_THREADS = SC_CONSUMERS + SC_PRODUCERS + 32;
+constexpr int SC_STAGES = 3;
+constexpr int SC_MAX_CHUNKS = 8;           // key chunks per group (pass-1 partial slots)
+constexpr int SC_GRID = 148;               // CTAs: one per B200 SM
+constexpr float SC_LAZY_LIMIT = 1048576.f;  // 2^20
 
 template <int D>
 struct ScoreSmem {
-  static constexpr uint32_t TILE = 128u * D * 2u;
-  static constexpr uint32_t CHUNK = 128u * 128u;
-  static constexpr int STAGES = 2;
-  static constexpr uint32_t FIX_OFF = 0;  // centroid tile
-  static constexpr uint32_t KP_OFF = FIX_OFF + TILE;
-  static constexpr uint32_t COL_OFF = KP_OFF + STAGES * TILE;  // pass 2: m[128], coef[128]
-  static constexpr uint32_t BAR_OFF = COL_OFF + 2u * 128u * 4u;
-  // CFULL, FULL[2], EMPTY[2], SFULL[2], SFREE[2], DRAIN
-  static constexpr uint32_t NBARS = 10;
+  static constexpr uint32_t CCHUNK = SC_ROWS * 128u;  // one 64-element column chunk, 256 rows
+  static constexpr uint32_t CENT_BYTES = (D / 64) * CCHUNK;
+  static constexpr uint32_t KCHUNK = 128u * 128u;
+  static constexpr uint32_t KTILE = (D / 64) * KCHUNK;
+  static constexpr uint32_t CENT_OFF = 0;
+  static constexpr uint32_t KP_OFF = CENT_OFF + CENT_BYTES;
+  static constexpr uint32_t COL_OFF = KP_OFF + SC_STAGES * KTILE;  // pass 2: m' per column
+  static constexpr uint32_t MERGE_OFF = COL_OFF + SC_ROWS * 4u;      // pass 1: (m, z) per row
+  static constexpr uint32_t BAR_OFF = MERGE_OFF + SC_ROWS * 8u;
+  // CFULL, CEMPTY, FULL[3], EMPTY[3], SFULL[2], SFREE[2], DRAIN
+  static constexpr uint32_t NBARS = 13;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NBARS * 8u;
   static constexpr uint32_t BYTES = MISC_OFF + 16u;
   static constexpr uint32_t ALLOC = BYTES + 1024u;
+  static_assert(KP_OFF % 1024u == 0, "swizzled tiles need 1024-byte alignment");
+  static_assert(ALLOC <= 232448u, "exceeds the 227 KB shared-memory limit per block");
 };
 
-enum { SB_CFULL = 0, SB_FULL0 = 1, SB_EMPTY0 = 3, SB_SFULL0 = 5, SB_SFREE0 = 7, SB_DRAIN = 9 };
+enum { SB_CFULL = 0, SB_CEMPTY = 1, SB_FULL0 = 2, SB_EMPTY0 = 5, SB_SFULL0 = 8, SB_SFREE0 = 10,
+       SB_DRAIN = 12 };
 
-// Two CTAs per SM (98 KB of shared memory and 256 TMEM columns each), so two consumer
-// warpgroups interleave their exp2 work on the MUFU units.
+// The work split shared by both passes (host and device compute it the same way).
+struct ScoreSplit {
+  int G;        // groups per head: ceil(nQ / 32)
+  int T;        // 128-key tiles per row: ceil(nK / 128)
+  int CT;       // tiles per chunk
+  int KC;       // chunks per group: ceil(T / CT) <= SC_MAX_CHUNKS
+  long long U;  // units = B*H * G * KC
+  int P;        // CTAs = min(U, SC_GRID)
+};
+
+inline ScoreSplit score_split(long long BH, long long nQ, long long nK) {
+  ScoreSplit s;
+  s.G = (int)((nQ + SC_QB - 1) / SC_QB);
+  s.T = (int)((nK + 127) / 128);
+  const int k = s.T < SC_MAX_CHUNKS ? s.T : SC_MAX_CHUNKS;
+  s.CT = (s.T + k - 1) / k;
+  s.KC = (s.T + s.CT - 1) / s.CT;
+  s.U = BH * s.G * s.KC;
+  s.P = (int)(s.U < SC_GRID ? s.U : SC_GRID);
+  return s;
+}
+
+// Sum over 32 logits of exp2(l * c + nm), four partial sums.
+AB_DEV float expsum32(const uint32_t* v, float c, float nm) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    s0 += fast_exp2(fmaf(__uint_as_float(v[k]), c, nm));
+    s1 += fast_exp2(fmaf(__uint_as_float(v[k + 1]), c, nm));
+    s2 += fast_exp2(fmaf(__uint_as_float(v[k + 2]), c, nm));
+    s3 += fast_exp2(fmaf(__uint_as_float(v[k + 3]), c, nm));
+  }
+  return (s0 + s1) + (s2 + s3);
+}
+
+// Adds a 32-logit chunk to the running (m, z) of one centroid row (see PASS 1 above).
+AB_DEV void online_chunk(uint32_t* v, float c, float& m, float& z) {
+  float acc = expsum32(v, c, -m);
+  if (!(acc <= SC_LAZY_LIMIT)) {  // first chunk (m = -inf), a maximum far above m, or NaN
+    float mt = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) mt = fmaxf(mt, __uint_as_float(v[k]));
+    const float mn = fmaxf(m, mt * c);
+    if (mn == -INFINITY) {
+      acc = 0.f;  // every key of the chunk is masked
+    } else {
+      z = (m == -INFINITY) ? 0.f : z * fast_exp2(m - mn);
+      m = mn;
+      acc = expsum32(v, c, -m);
+    }
+  }
+  z += acc;
+}
+
 template <int D, int PASS>
-__global__ void __launch_bounds__(SCT_THREADS, 2) score_tc_kernel(SelectArgs a, uint64_t timeout_ns) {
+__global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, ScoreSplit sp,
+                                                              uint64_t timeout_ns) {
   using L = ScoreSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -314,28 +394,31 @@ __global__ void __launch_bounds__(SCT_THREADS, 2) score_tc_kernel(SelectArgs a, 
   uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF);
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF + 4);
-  float2* col_mc = (float2*)(smem + L::COL_OFF);  // pass 2: (m, w/Z) per centroid column
+  float* col_m = (float*)(smem + L::COL_OFF);
+  float2* merge = (float2*)(smem + L::MERGE_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int groups = (a.nQ + 15) / 16;
-  const int bh = blockIdx.x / groups;
-  const int g = blockIdx.x - bh * groups;
-  const int T = (a.nK + 127) / 128;
+  // this CTA's run of units [u0, u1)
+  const long long u0 = (long long)blockIdx.x * sp.U / gridDim.x;
+  const long long u1 = (long long)(blockIdx.x + 1) * sp.U / gridDim.x;
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(&bars[SB_CFULL], 128);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars[SB_FULL0 + b], 128);
+    mbar_init(&bars[SB_CFULL], SC_PRODUCERS);
+    mbar_init(&bars[SB_CEMPTY], 1);
+    for (int b = 0; b < SC_STAGES; ++b) {
+      mbar_init(&bars[SB_FULL0 + b], SC_PRODUCERS);
       mbar_init(&bars[SB_EMPTY0 + b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[SB_SFULL0 + b], 1);
-      mbar_init(&bars[SB_SFREE0 + b], 128);
+      mbar_init(&bars[SB_SFREE0 + b], SC_CONSUMERS);
     }
     mbar_init(&bars[SB_DRAIN], 1);
     fence_mbar_init();
   }
-  if (warp == 8) {
-    tmem_alloc(tmem_slot, 256);
+  if (warp == 18) {
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -343,155 +426,227 @@ __global__ void __launch_bounds__(SCT_THREADS, 2) score_tc_kernel(SelectArgs a, 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 4 && warp < 8) {
+  // Segments: maximal runs of units of one group.  For a segment starting at unit u:
+  // group gi = u / KC, tiles [k0 * CT, min(T, (k1 + 1) * CT)) for its chunks k0..k1.
+  auto segment = [&](long long u, long long& unext, long long& gi, int& k0, int& t0, int& t1) {
+    gi = u / sp.KC;
+    k0 = (int)(u - gi * sp.KC);
+    const long long uend = min(u1, (gi + 1) * (long long)sp.KC);
+    t0 = k0 * sp.CT;
+    t1 = (int)min((long long)sp.T, (uend - gi * sp.KC) * (long long)sp.CT);
+    unext = uend;
+  };
+
+  if (warp >= 16 && warp < 18) {
     // ---------------------------------------------------------------- producers
-    const int p = tid - 128, u = p & 15, rsub = p >> 4;
-    constexpr int UNITS = D / 8;
-    for (int r = rsub; r < 128; r += 8) {  // centroid rows: 16 query blocks x 8 slots
-      if (u < UNITS) {
-        const int qb = g * 16 + (r >> 3);
-        const bool ok = qb < a.nQ;
-        const uint16_t* src = a.cent + (((size_t)bh * a.nQ + (ok ? qb : 0)) * CMAX + (r & 7)) * D + u * 8;
-        cp_async_16(sbase + L::FIX_OFF + (u >> 3) * L::CHUNK + sw128_off(r, u & 7), src, ok ? 16u : 0u);
+    constexpr int UNITS = D / 8;           // 16-byte units per row
+    constexpr int RSTEP = SC_PRODUCERS / UNITS;
+    const int p = tid - SC_CONSUMERS, u = p % UNITS, rsub = p / UNITS;
+    long long it = 0;  // tiles of this CTA so far
+    int sg = 0;        // segments so far
+    bool ok = true;
+    for (long long uu = u0; uu < u1 && ok; ++sg) {
+      long long unext, gi;
+      int k0, t0, t1;
+      segment(uu, unext, gi, k0, t0, t1);
+      uu = unext;
+      if (sg > 0 && !mbar_wait(&bars[SB_CEMPTY], (sg - 1) & 1, abort_flag, timeout_ns)) break;
+      const long long bh = gi / sp.G;
+      const int qb0 = (int)(gi - bh * sp.G) * SC_QB;
+      for (int r = rsub; r < SC_ROWS; r += RSTEP) {  // centroid rows: 32 query blocks x 8
+        const int qb = qb0 + (r >> 3);
+        const bool in = qb < a.nQ;
+        const uint16_t* src = a.cent + (((size_t)bh * a.nQ + (in ? qb : 0)) * CMAX + (r & 7)) * D + u * 8;
+        cp_async_16(sbase + L::CENT_OFF + (u >> 3) * L::CCHUNK + sw128_off(r, u & 7), src, in ? 16u : 0u);
       }
-    }
-    mbar_arrive_cpasync(&bars[SB_CFULL]);
-    const uint16_t* kp = a.Kp + (size_t)bh * a.nK * D;
-    for (int t = 0; t < T; ++t) {
-      const int st = t & 1;
-      if (t >= 2 && !mbar_wait(&bars[SB_EMPTY0 + st], ((t >> 1) - 1) & 1, abort_flag, timeout_ns)) break;
-      const uint32_t dst = sbase + L::KP_OFF + st * L::TILE;
-      for (int r = rsub; r < 128; r += 8) {
-        if (u < UNITS) {
-          const int j = t * 128 + r;
-          const bool ok = j < a.nK;
-          cp_async_16(dst + (u >> 3) * L::CHUNK + sw128_off(r, u & 7),
-                      kp + (size_t)(ok ? j : 0) * D + u * 8, ok ? 16u : 0u);
+      mbar_arrive_cpasync(&bars[SB_CFULL]);
+      const uint16_t* kp = a.Kp + (size_t)bh * a.nK * D;
+      for (int t = t0; t < t1; ++t, ++it) {
+        const int st = (int)(it % SC_STAGES);
+        if (it >= SC_STAGES &&
+            !mbar_wait(&bars[SB_EMPTY0 + st], (int)((it / SC_STAGES - 1) & 1), abort_flag, timeout_ns)) {
+          ok = false;
+          break;
         }
+        const uint32_t dst = sbase + L::KP_OFF + st * L::KTILE;
+        for (int r = rsub; r < 128; r += RSTEP) {
+          const int j = t * 128 + r;
+          const bool in = j < a.nK;
+          cp_async_16(dst + (u >> 3) * L::KCHUNK + sw128_off(r, u & 7),
+                      kp + (size_t)(in ? j : 0) * D + u * 8, in ? 16u : 0u);
+        }
+        mbar_arrive_cpasync(&bars[SB_FULL0 + st]);
       }
-      mbar_arrive_cpasync(&bars[SB_FULL0 + st]);
     }
     cp_async_wait_all();
-  } else if (warp == 8) {
+  } else if (warp == 18) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, 0, 0);
-      bool ok = mbar_wait(&bars[SB_CFULL], 0, abort_flag, timeout_ns);
-      for (int t = 0; t < T && ok; ++t) {
-        const int st = t & 1;
-        ok = mbar_wait(&bars[SB_FULL0 + st], (t >> 1) & 1, abort_flag, timeout_ns);
-        if (ok && t >= 2) ok = mbar_wait(&bars[SB_SFREE0 + st], ((t >> 1) - 1) & 1, abort_flag, timeout_ns);
-        if (!ok) break;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t cbase = sbase + L::FIX_OFF;
-        const uint32_t kbase = sbase + L::KP_OFF + st * L::TILE;
+      constexpr uint32_t IDESC1 = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC2 = idesc_bf16_f32(128, SC_ROWS, 0, 0);
+      long long it = 0;
+      int sg = 0;
+      bool ok = true;
+      for (long long uu = u0; uu < u1 && ok; ++sg) {
+        long long unext, gi;
+        int k0, t0, t1;
+        segment(uu, unext, gi, k0, t0, t1);
+        uu = unext;
+        if (!(ok = mbar_wait(&bars[SB_CFULL], sg & 1, abort_flag, timeout_ns))) break;
+        for (int t = t0; t < t1; ++t, ++it) {
+          const int st = (int)(it % SC_STAGES), b = (int)(it & 1);
+          ok = mbar_wait(&bars[SB_FULL0 + st], (int)((it / SC_STAGES) & 1), abort_flag, timeout_ns);
+          if (ok && it >= 2) ok = mbar_wait(&bars[SB_SFREE0 + b], (int)(((it >> 1) - 1) & 1), abort_flag, timeout_ns);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint32_t cbase = sbase + L::CENT_OFF;
+          const uint32_t kbase = sbase + L::KP_OFF + st * L::KTILE;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::CHUNK + (kk & 3) * 32;
-          const uint64_t dc = sdesc_sw128(cbase + off, 16, 1024);
-          const uint64_t dk = sdesc_sw128(kbase + off, 16, 1024);
-          if (PASS == 1) umma_f16_ss(tmem + st * 128, dc, dk, IDESC, kk > 0 ? 1u : 0u);
-          else umma_f16_ss(tmem + st * 128, dk, dc, IDESC, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk & 3) * 32;
+            const uint64_t dk = sdesc_sw128(kbase + (kk >> 2) * L::KCHUNK + ko, 16, 1024);
+            const uint64_t dc = sdesc_sw128(cbase + (kk >> 2) * L::CCHUNK + ko, 16, 1024);
+            if (PASS == 1) {
+              umma_f16_ss(tmem + b * 256, dc, dk, IDESC1, kk > 0 ? 1u : 0u);
+              const uint64_t dc1 = sdesc_sw128(cbase + (kk >> 2) * L::CCHUNK + 128u * 128u + ko, 16, 1024);
+              umma_f16_ss(tmem + b * 256 + 128, dc1, dk, IDESC1, kk > 0 ? 1u : 0u);
+            } else {
+              umma_f16_ss(tmem + b * 256, dk, dc, IDESC2, kk > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&bars[SB_SFULL0 + b]);
+          umma_commit(&bars[SB_EMPTY0 + st]);
         }
-        umma_commit(&bars[SB_SFULL0 + st]);
-        umma_commit(&bars[SB_EMPTY0 + st]);
+        umma_commit(&bars[SB_CEMPTY]);  // the centroid buffer is free once these MMAs end
       }
       umma_commit(&bars[SB_DRAIN]);
       mbar_wait(&bars[SB_DRAIN], 0, abort_flag, timeout_ns);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- consumers (warps 0-3)
-    const int r = tid;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    if (PASS == 2) {  // per-column constants: column r = (query block r>>3, slot r&7)
-      const int qb = g * 16 + (r >> 3);
-      float mm = 0.f, cf = 0.f;
-      if (qb < a.nQ) {
-        const size_t crow = ((size_t)bh * a.nQ + qb) * CMAX + (r & 7);
-        const float Z = a.stats[crow * 2 + 1];
-        mm = a.stats[crow * 2];
-        cf = (Z > 0.f) ? a.w[crow] / Z : 0.f;
-        if (!(mm > -INFINITY)) { mm = 0.f; cf = 0.f; }
-      }
-      col_mc[r] = make_float2(mm, cf);
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 consumer warps only
-    }
-    float m = -INFINITY, z = 0.f;
+    // ---------------------------------------------------------------- consumers (warps 0-15)
+    const int q = warp & 3, sub = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float c = a.scale_log2;
+    long long it = 0;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int st = t & 1;
-      ok = mbar_wait(&bars[SB_SFULL0 + st], (t >> 1) & 1, abort_flag, timeout_ns);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t sadr = tmem + st * 128 + lane_off;
-      if (PASS == 1) {
-        // online max / sum over 32-column chunks (keeps 32 values live)
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(sadr + c0, v);
-          tmem_wait_ld();
-          float mt = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float l = (t * 128 + c0 + c < a.nK) ? __uint_as_float(v[c]) * a.scale_log2 : -INFINITY;
-            v[c] = __float_as_uint(l);
-            mt = fmaxf(mt, l);
+    for (long long uu = u0; uu < u1;) {
+      long long unext, gi;
+      int k0, t0, t1;
+      segment(uu, unext, gi, k0, t0, t1);
+      uu = unext;
+      const long long bh = gi / sp.G;
+      const int qb0 = (int)(gi - bh * sp.G) * SC_QB;
+      if (PASS == 2) {
+        // the column constants m' of this group (every consumer passes both barriers)
+        asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
+        if (tid < SC_ROWS) {
+          const int qb = qb0 + (tid >> 3);
+          float mp = INFINITY;
+          if (qb < a.nQ) {
+            const float2* sl = (const float2*)a.stats + ((size_t)gi * SC_ROWS + tid) * SC_MAX_CHUNKS;
+            float M = -INFINITY, Z = 0.f;
+            for (int k = 0; k < sp.KC; ++k) M = fmaxf(M, sl[k].x);
+            if (M > -INFINITY)
+              for (int k = 0; k < sp.KC; ++k) {
+                const float2 mz = sl[k];
+                if (mz.x > -INFINITY) Z += mz.y * fast_exp2(mz.x - M);
+              }
+            const float w = a.w[((size_t)bh * a.nQ + qb) * CMAX + (tid & 7)];
+            if (w > 0.f && Z > 0.f && M > -INFINITY) mp = M + (log2f(Z) - log2f(w));
           }
-          if (mt > m) {
-            z = (m == -INFINITY) ? 0.f : z * fast_exp2(m - mt);
-            m = mt;
-          }
-          float acc = 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) acc += fast_exp2(__uint_as_float(v[c]) - m);
-          z += acc;
+          col_m[tid] = mp;
         }
-        tc_fence_before();
-        mbar_arrive(&bars[SB_SFREE0 + st]);
-      } else {
-        const int j = t * 128 + r;
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {  // 4 query blocks per TMEM load
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(sadr + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              // re-read per tile (volatile): hoisting all 128 columns would need 256 registers
-              float mm, cf;
-              asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
-                           : "=f"(mm), "=f"(cf)
-                           : "r"(smem_u32(col_mc + c0 + q * 8 + c)));
-              acc = fmaf(cf, fast_exp2(fmaf(__uint_as_float(v[q * 8 + c]), a.scale_log2, -mm)), acc);
-            }
-            const int qb = g * 16 + (c0 >> 3) + q;
-            if (j < a.nK && qb < a.nQ) a.S[((size_t)bh * a.nQ + qb) * a.nK + j] = acc;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&bars[SB_SFREE0 + st]);
+        asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
       }
-    }
-    if (PASS == 1 && ok) {
-      const int qb = g * 16 + (r >> 3);
-      if (qb < a.nQ) {
-        const size_t crow = ((size_t)bh * a.nQ + qb) * CMAX + (r & 7);
-        a.stats[crow * 2] = m;
-        a.stats[crow * 2 + 1] = z;
+      const int h = sub >> 1, ch = sub & 1;  // pass 1: centroid half, key half
+      float m = -INFINITY, z = 0.f;
+      for (int t = t0; t < t1; ++t, ++it) {
+        const int b = (int)(it & 1);
+        if (ok) ok = mbar_wait(&bars[SB_SFULL0 + b], (int)((it >> 1) & 1), abort_flag, timeout_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          if (PASS == 1) {
+            uint32_t v[64];
+            const uint32_t col = b * 256 + h * 128 + ch * 64;
+            tmem_ld_32x32b_x32(tmem + lane_off + col, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_ld_32x32b_x32(tmem + lane_off + col + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars[SB_SFREE0 + b]);
+            const int jb = t * 128 + ch * 64;  // key of v[0]
+            if (jb + 64 > a.nK) {              // the ragged last tile: mask keys >= nK
+#pragma unroll
+              for (int k = 0; k < 64; ++k)
+                if (jb + k >= a.nK) v[k] = __float_as_uint(-INFINITY);
+            }
+            online_chunk(v, c, m, z);
+            online_chunk(v + 32, c, m, z);
+          } else {
+            // two rounds of 32 columns (4 query blocks each); TMEM is released after the second
+            const int j = t * 128 + q * 32 + lane;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(tmem + lane_off + b * 256 + sub * 64 + half * 32, v);
+              tmem_wait_ld();
+              if (half == 1) {
+                tc_fence_before();
+                mbar_arrive(&bars[SB_SFREE0 + b]);
+              }
+#pragma unroll
+              for (int qq = 0; qq < 4; ++qq) {
+                const int cb = sub * 64 + half * 32 + qq * 8;  // first column of this query block
+                float mp[8];
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(mp[0]), "=f"(mp[1]), "=f"(mp[2]), "=f"(mp[3])
+                             : "r"(smem_u32(col_m + cb)));
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(mp[4]), "=f"(mp[5]), "=f"(mp[6]), "=f"(mp[7])
+                             : "r"(smem_u32(col_m + cb + 4)));
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < 8; k += 2) {
+                  s0 += fast_exp2(fmaf(__uint_as_float(v[qq * 8 + k]), c, -mp[k]));
+                  s1 += fast_exp2(fmaf(__uint_as_float(v[qq * 8 + k + 1]), c, -mp[k + 1]));
+                }
+                const int qb = qb0 + (cb >> 3);
+                if (j < a.nK && qb < a.nQ) a.S[((size_t)bh * a.nQ + qb) * a.nK + j] = s0 + s1;
+              }
+            }
+          }
+        }
+        if (PASS == 1 && (t + 1 == t1 || (t + 1) % sp.CT == 0)) {
+          // end of key chunk t / CT: merge the two key halves of each row into its slot.
+          // Each chunk's (m, z) depends only on its own keys, so S does not depend on how
+          // the units were dealt out to CTAs.
+          asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
+          const int row = h * 128 + q * 32 + lane;
+          if (ch == 1) merge[row] = make_float2(m, z);
+          asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
+          if (ch == 0 && ok) {
+            const float2 o = merge[row];
+            const float M = fmaxf(m, o.x);
+            float Z = 0.f;
+            if (M > -INFINITY) {
+              if (m > -INFINITY) Z += z * fast_exp2(m - M);
+              if (o.x > -INFINITY) Z += o.y * fast_exp2(o.x - M);
+            }
+            ((float2*)a.stats)[((size_t)gi * SC_ROWS + row) * SC_MAX_CHUNKS + t / sp.CT] = make_float2(M, Z);
+          }
+          m = -INFINITY;
+          z = 0.f;
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 18) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
