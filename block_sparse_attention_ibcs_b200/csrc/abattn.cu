@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <cudaTypedefs.h>
+
 #include "abattn.h"
 #include "attn.cuh"
 #include "common.cuh"
@@ -86,6 +88,34 @@ ab_status launch_status() {
   return AB_OK;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (the library
+// does not link libcuda directly).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return (PFN_cuTensorMapEncodeTiled_v12000)f;
+  }();
+  return fn;
+}
+
+// Tensor map of a bf16 array [z][y][x] (x contiguous, x = d elements) read in boxes of
+// 64 x box_y x 1 with the 128-byte swizzle; out-of-range rows read as zeros.
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z, uint32_t box_y) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {x, y, z};
+  const cuuint64_t strides[2] = {x * 2, x * y * 2};  // bytes, dimensions 1 and 2
+  const cuuint32_t box[3] = {64, box_y, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, const Workspace& ws,
                      int8_t* labels, cudaStream_t st) {
@@ -117,8 +147,14 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
       cudaFuncSetAttribute(score_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SL::ALLOC) != cudaSuccess)
     return launch_status();
-  score_kernel<D, 1><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, kDefaultTimeoutNs);
-  score_kernel<D, 2><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, kDefaultTimeoutNs);
+  CUtensorMap tm_kp, tm_cent;
+  if (!make_tmap_3d(&tm_kp, ws.Kp, D, (uint64_t)d.nK, (uint64_t)d.BH, 128) ||
+      !make_tmap_3d(&tm_cent, ws.cent, D, (uint64_t)d.nQ * CMAX, (uint64_t)d.BH, SC_ROWS)) {
+    fprintf(stderr, "abattn: cannot encode the selector's tensor maps\n");
+    return AB_ERR_CUDA;
+  }
+  score_kernel<D, 1><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, tm_kp, tm_cent, kDefaultTimeoutNs);
+  score_kernel<D, 2><<<sp.P, SC_THREADS, SL::ALLOC, st>>>(a, sp, tm_kp, tm_cent, kDefaultTimeoutNs);
   return launch_status();
 }
 

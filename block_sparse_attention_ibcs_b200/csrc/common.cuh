@@ -5,6 +5,7 @@
 // device status word and exact fp64 -> bf16 rounding.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -56,6 +57,63 @@ AB_DEV float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ------------------------------------------------------------------ packed fp32 pairs
+//
+// sm_100 executes fp32 add and fma on register pairs (.f32x2), one instruction per pair.
+
+AB_DEV uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+AB_DEV float2 f2_unpack(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+AB_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+AB_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (so that part of the exponentials stays off the MUFU).
+// Range reduction x = j + f with j = round(x) (the 1.5 * 2^23 rounding constant) and
+// |f| <= 1/2; 2^f by a degree-5 polynomial; 2^j added into the exponent field.  The
+// coefficients are this library's own fit: Lawson's iteratively reweighted least squares
+// for minimax relative error of 2^f on [-1/2, 1/2], rounded to fp32; evaluated by Horner
+// in fp32 the maximum relative error is 2.4e-7 (ex2.approx: about 2^-22).  x is clamped
+// to [-126, 127]; below -126 the result is a value under 2^-125 instead of the flushed 0.
+constexpr float EXP2P_C0 = 1.0000001192092896f;
+constexpr float EXP2P_C1 = 0.6931469440460205f;
+constexpr float EXP2P_C2 = 0.24022120237350464f;
+constexpr float EXP2P_C3 = 0.05550713092088699f;
+constexpr float EXP2P_C4 = 0.009675541892647743f;
+constexpr float EXP2P_C5 = 0.001327647129073739f;
+constexpr float EXP2P_ROUND = 12582912.0f;  // 1.5 * 2^23
+
+AB_DEV uint64_t exp2_poly_x2(float x0, float x1) {
+  x0 = fminf(fmaxf(x0, -126.f), 127.f);
+  x1 = fminf(fmaxf(x1, -126.f), 127.f);
+  const uint64_t X = f2_pack(x0, x1);
+  const uint64_t T = f2_add(X, f2_pack(EXP2P_ROUND, EXP2P_ROUND));  // its low bits hold j
+  const uint64_t J = f2_add(T, f2_pack(-EXP2P_ROUND, -EXP2P_ROUND));
+  const uint64_t F = f2_fma(J, f2_pack(-1.f, -1.f), X);  // x - j, exact
+  uint64_t P = f2_fma(f2_pack(EXP2P_C5, EXP2P_C5), F, f2_pack(EXP2P_C4, EXP2P_C4));
+  P = f2_fma(P, F, f2_pack(EXP2P_C3, EXP2P_C3));
+  P = f2_fma(P, F, f2_pack(EXP2P_C2, EXP2P_C2));
+  P = f2_fma(P, F, f2_pack(EXP2P_C1, EXP2P_C1));
+  P = f2_fma(P, F, f2_pack(EXP2P_C0, EXP2P_C0));
+  const float2 t = f2_unpack(T), pv = f2_unpack(P);
+  return f2_pack(__uint_as_float(__float_as_uint(pv.x) + (__float_as_uint(t.x) << 23)),
+                 __uint_as_float(__float_as_uint(pv.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // ------------------------------------------------------------------ mbarriers
@@ -122,6 +180,34 @@ AB_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint6
       return false;
     }
   }
+}
+
+// Arrive on `bar` (one of its expected arrivals) and add `bytes` to the transaction
+// count that the bulk copies signalling it must complete.
+AB_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait that ignores the CTA's abort flag (used on the way out, to let copies that
+// are already in flight land before the CTA exits).  Returns whether the phase completed.
+AB_DEV bool mbar_wait_quiet(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity))
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  return true;
+}
+
+// ------------------------------------------------------------------ TMA (tiled, no multicast)
+
+// 3-D tiled bulk copy global -> shared of the box at (x, y, z) of `tmap`, completing `bytes`
+// of transactions on `bar`.  x * element size must be a multiple of 16 bytes.
+AB_DEV void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"((uint64_t)tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------------ cp.async
@@ -220,6 +306,19 @@ AB_DEV void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
+      : "memory");
+}
+// tcgen05.wait::ld that also names the destination registers of the loads it waits for,
+// so the compiler cannot move a use of them above the wait.
+AB_DEV void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
       : "memory");
 }
 AB_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

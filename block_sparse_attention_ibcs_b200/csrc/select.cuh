@@ -276,32 +276,42 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
 // The page's batched scoring ("premises & limits": query/KV blocks scored as batched
 // matrix operations) as two persistent tensor-core streaming passes.  A group is 32 query
 // blocks of one head (256 centroid rows); its key axis is cut into chunks of whole
-// 128-key tiles.  The (group, chunk) units are dealt out in order, in equal contiguous
-// runs, to one CTA per SM; a CTA walks its run as segments (consecutive units of one
-// group), loading the group's centroids once per segment.
+// 128-key tiles.  The (group, chunk) units, numbered head by head, are dealt out
+// round-robin to one CTA per SM, so the CTAs running at any moment work on about one
+// head and share its pooled keys in L2 (all heads' pooled keys together exceed L2 at the
+// Wan2.1-14B shape).  A CTA loads a unit's centroids, then streams the chunk's key tiles;
+// the first key tiles of the next unit are requested before its centroids, so the
+// centroid reload overlaps the end of the previous unit.
 //   PASS 1: D[centroid row, key] = C Kp^T for the two 128-row halves of the centroids
 //           (A = centroids, B = key tile, both K-major, N = 128).  Each thread keeps a
 //           running reference m and sum z of exp2(logit - m) for one centroid row over
-//           64 of the tile's keys.  m is raised lazily: a 32-key chunk whose sum stays
+//           the unit's keys.  m is raised lazily: a 32-key chunk whose sum stays
 //           below 2^20 is accepted as it is (a term can then exceed 1 by at most 2^20,
 //           far from fp32 overflow); otherwise the chunk's maximum is taken and z rescaled.
-//           At the end of each key chunk the two key halves of a row are merged and the
-//           chunk's (m, z) is stored in its own slot; pass 2 merges a row's slots in chunk
-//           order, so S does not depend on how the units were dealt out to CTAs.
+//           At the end of each unit the two groups' (m, z) of a row are merged and stored
+//           in the slot of the unit's key chunk; pass 2 merges a row's slots in chunk order, so S does not depend on how
+//           the units were dealt out to CTAs.
 //   PASS 2: D[key, centroid column] = Kp C^T (A = key tile, B = all 256 centroid rows,
 //           N = 256), so thread j owns one KV block and sums exp2(logit - m'_c) over the
-//           8 columns of each of its 8 query blocks in registers, where the share and
+//           8 columns of each of its 16 query blocks in registers, where the share and
 //           the softmax normaliser are folded into one constant per column:
 //           w_c exp2(l - m_c) / Z_c = exp2(l - (m_c + log2 Z_c - log2 w_c)).
 //           S rows are stored coalesced.
-// Roles: warps 0-15 consume TMEM (lane quadrant = warp % 4), warps 16-17 stream tiles with
-// cp.async (3 stages), warp 18 allocates 512 TMEM columns and issues the MMAs.
+// Roles: warps 0-15 consume TMEM in two groups that alternate tiles (group g = warp / 8
+// takes the unit's tiles t0 + g, t0 + g + 2, ..., which the MMAs put in TMEM buffer g), so one group's exponentials cover the other's TMEM
+// loads; in a group, lane quadrant = warp % 4 and each thread reads 128 columns of its
+// tile in four 32-column chunks.  One thread of warp 16 streams the centroids and the key tiles with TMA (3-D
+// tiled boxes with the 128-byte swizzle the MMA descriptors expect; rows past the head's
+// end are filled with zeros), 3 stages deep; warp 17 allocates 512 TMEM columns and one of
+// its threads issues the MMAs.
 
 constexpr int SC_QB = 32;                  // query blocks per group
 constexpr int SC_ROWS = SC_QB * CMAX;      // 256 centroid rows per group
-constexpr int SC_CONSUMERS = 512;          // warps 0-15
-constexpr int SC_PRODUCERS = 64;           // warps 16-17
-constexpr int SC_THREADS = SC_CONSUMERS + SC_PRODUCERS + 32;
+constexpr int SC_CONSUMERS = 512;          // warps 0-15: two groups of 8
+constexpr int SC_GROUP = 256;              // consumers of one TMEM buffer
+constexpr int SC_PRODUCER_WARP = 16;       // TMA producer
+constexpr int SC_MMA_WARP = 17;            // TMEM allocation, MMA issue
+constexpr int SC_THREADS = SC_CONSUMERS + 64;
 constexpr int SC_STAGES = 3;
 constexpr int SC_MAX_CHUNKS = 8;           // key chunks per group (pass-1 partial slots)
 constexpr int SC_GRID = 148;               // CTAs: one per B200 SM
@@ -352,41 +362,54 @@ inline ScoreSplit score_split(long long BH, long long nQ, long long nK) {
   return s;
 }
 
-// Sum over 32 logits of exp2(l * c + nm), four partial sums.
-AB_DEV float expsum32(const uint32_t* v, float c, float nm) {
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+// Exponentials per 32-logit chunk (pass 1) and per 8-column query block (pass 2) that go
+// to the FMA-pipe polynomial instead of the MUFU, in pairs: of 16 and of 4 pairs.
+#ifndef SC_POLY_PAIRS1
+#define SC_POLY_PAIRS1 2
+#endif
+#ifndef SC_POLY_PAIRS2
+#define SC_POLY_PAIRS2 0
+#endif
+
+// Sum over 32 logits of exp2(l * c + nm), in packed pairs; the first NP of the 16 pairs use
+// the polynomial exp2, the others the MUFU.  Four independent partial sums.
+template <int NP>
+AB_DEV float expsum32(const uint32_t (&v)[32], float c, float nm) {
+  const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(nm, nm);
+  uint64_t a[4] = {0, 0, 0, 0};  // (0.f, 0.f)
 #pragma unroll
-  for (int k = 0; k < 32; k += 4) {
-    s0 += fast_exp2(fmaf(__uint_as_float(v[k]), c, nm));
-    s1 += fast_exp2(fmaf(__uint_as_float(v[k + 1]), c, nm));
-    s2 += fast_exp2(fmaf(__uint_as_float(v[k + 2]), c, nm));
-    s3 += fast_exp2(fmaf(__uint_as_float(v[k + 3]), c, nm));
+  for (int i = 0; i < 16; ++i) {
+    const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2));
+    const uint64_t e = (i < NP) ? exp2_poly_x2(x.x, x.y) : f2_pack(fast_exp2(x.x), fast_exp2(x.y));
+    a[i & 3] = f2_add(a[i & 3], e);
   }
-  return (s0 + s1) + (s2 + s3);
+  const float2 s = f2_unpack(f2_add(f2_add(a[0], a[1]), f2_add(a[2], a[3])));
+  return s.x + s.y;
 }
 
-// Adds a 32-logit chunk to the running (m, z) of one centroid row (see PASS 1 above).
-AB_DEV void online_chunk(uint32_t* v, float c, float& m, float& z) {
-  float acc = expsum32(v, c, -m);
-  if (!(acc <= SC_LAZY_LIMIT)) {  // first chunk (m = -inf), a maximum far above m, or NaN
+// Adds a chunk of 32 logits to the running (m, z) of one centroid row (see PASS 1 above).
+AB_DEV void online_chunk(const uint32_t (&v)[32], float c, float& m, float& z) {
+  float acc = expsum32<SC_POLY_PAIRS1>(v, c, -m);
+  if (m == -INFINITY || !(acc <= SC_LAZY_LIMIT)) {  // first chunk, a maximum far above m, or NaN
     float mt = -INFINITY;
 #pragma unroll
     for (int k = 0; k < 32; ++k) mt = fmaxf(mt, __uint_as_float(v[k]));
     const float mn = fmaxf(m, mt * c);
     if (mn == -INFINITY) {
-      acc = 0.f;  // every key of the chunk is masked
+      acc = 0.f;  // every key is masked
     } else {
       z = (m == -INFINITY) ? 0.f : z * fast_exp2(m - mn);
       m = mn;
-      acc = expsum32(v, c, -m);
+      acc = expsum32<0>(v, c, -m);
     }
   }
   z += acc;
 }
 
 template <int D, int PASS>
-__global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, ScoreSplit sp,
-                                                              uint64_t timeout_ns) {
+__global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(
+    SelectArgs a, ScoreSplit sp, const __grid_constant__ CUtensorMap tm_kp,
+    const __grid_constant__ CUtensorMap tm_cent, uint64_t timeout_ns) {
   using L = ScoreSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -398,26 +421,22 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, Scor
   float2* merge = (float2*)(smem + L::MERGE_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // this CTA's run of units [u0, u1)
-  const long long u0 = (long long)blockIdx.x * sp.U / gridDim.x;
-  const long long u1 = (long long)(blockIdx.x + 1) * sp.U / gridDim.x;
-
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(&bars[SB_CFULL], SC_PRODUCERS);
+    mbar_init(&bars[SB_CFULL], 1);
     mbar_init(&bars[SB_CEMPTY], 1);
     for (int b = 0; b < SC_STAGES; ++b) {
-      mbar_init(&bars[SB_FULL0 + b], SC_PRODUCERS);
+      mbar_init(&bars[SB_FULL0 + b], 1);
       mbar_init(&bars[SB_EMPTY0 + b], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[SB_SFULL0 + b], 1);
-      mbar_init(&bars[SB_SFREE0 + b], SC_CONSUMERS);
+      mbar_init(&bars[SB_SFREE0 + b], SC_GROUP);
     }
     mbar_init(&bars[SB_DRAIN], 1);
     fence_mbar_init();
   }
-  if (warp == 18) {
+  if (warp == SC_MMA_WARP) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -426,78 +445,80 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, Scor
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Segments: maximal runs of units of one group.  For a segment starting at unit u:
-  // group gi = u / KC, tiles [k0 * CT, min(T, (k1 + 1) * CT)) for its chunks k0..k1.
-  auto segment = [&](long long u, long long& unext, long long& gi, int& k0, int& t0, int& t1) {
-    gi = u / sp.KC;
-    k0 = (int)(u - gi * sp.KC);
-    const long long uend = min(u1, (gi + 1) * (long long)sp.KC);
-    t0 = k0 * sp.CT;
-    t1 = (int)min((long long)sp.T, (uend - gi * sp.KC) * (long long)sp.CT);
-    unext = uend;
+  // Units of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...  Unit un is chunk
+  // k = un % KC of group gi = un / KC: tiles [k * CT, min(T, (k + 1) * CT)).
+  auto unit = [&](long long un, long long& gi, int& t0, int& t1) {
+    gi = un / sp.KC;
+    const int k = (int)(un - gi * sp.KC);
+    t0 = k * sp.CT;
+    t1 = min(sp.T, t0 + sp.CT);
   };
 
-  if (warp >= 16 && warp < 18) {
-    // ---------------------------------------------------------------- producers
-    constexpr int UNITS = D / 8;           // 16-byte units per row
-    constexpr int RSTEP = SC_PRODUCERS / UNITS;
-    const int p = tid - SC_CONSUMERS, u = p % UNITS, rsub = p / UNITS;
-    long long it = 0;  // tiles of this CTA so far
-    int sg = 0;        // segments so far
-    bool ok = true;
-    for (long long uu = u0; uu < u1 && ok; ++sg) {
-      long long unext, gi;
-      int k0, t0, t1;
-      segment(uu, unext, gi, k0, t0, t1);
-      uu = unext;
-      if (sg > 0 && !mbar_wait(&bars[SB_CEMPTY], (sg - 1) & 1, abort_flag, timeout_ns)) break;
-      const long long bh = gi / sp.G;
-      const int qb0 = (int)(gi - bh * sp.G) * SC_QB;
-      for (int r = rsub; r < SC_ROWS; r += RSTEP) {  // centroid rows: 32 query blocks x 8
-        const int qb = qb0 + (r >> 3);
-        const bool in = qb < a.nQ;
-        const uint16_t* src = a.cent + (((size_t)bh * a.nQ + (in ? qb : 0)) * CMAX + (r & 7)) * D + u * 8;
-        cp_async_16(sbase + L::CENT_OFF + (u >> 3) * L::CCHUNK + sw128_off(r, u & 7), src, in ? 16u : 0u);
-      }
-      mbar_arrive_cpasync(&bars[SB_CFULL]);
-      const uint16_t* kp = a.Kp + (size_t)bh * a.nK * D;
-      for (int t = t0; t < t1; ++t, ++it) {
+  if (warp == SC_PRODUCER_WARP) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      long long it = 0;  // tiles of this CTA so far
+      int sg = 0;        // units so far
+      bool ok = true;
+      auto load_tile = [&](int bh, int t) -> bool {
         const int st = (int)(it % SC_STAGES);
         if (it >= SC_STAGES &&
-            !mbar_wait(&bars[SB_EMPTY0 + st], (int)((it / SC_STAGES - 1) & 1), abort_flag, timeout_ns)) {
-          ok = false;
-          break;
+            !mbar_wait(&bars[SB_EMPTY0 + st], (int)((it / SC_STAGES - 1) & 1), abort_flag, timeout_ns))
+          return false;
+        mbar_arrive_expect_tx(&bars[SB_FULL0 + st], L::KTILE);
+#pragma unroll
+        for (int ck = 0; ck < D / 64; ++ck)  // keys t*128 .. t*128 + 127 of head bh
+          tma_load_3d(sbase + L::KP_OFF + st * L::KTILE + ck * L::KCHUNK, &tm_kp, ck * 64, t * 128, bh,
+                      &bars[SB_FULL0 + st]);
+        ++it;
+        return true;
+      };
+      for (long long un = blockIdx.x; un < sp.U && ok; un += gridDim.x, ++sg) {
+        long long gi;
+        int t0, t1;
+        unit(un, gi, t0, t1);
+        const int bh = (int)(gi / sp.G);
+        const int qb0 = (int)(gi - (long long)bh * sp.G) * SC_QB;
+        int t = t0;
+        if (sg > 0) {  // the first key tiles, then wait until the centroid buffer is free
+          for (; t < min(t1, t0 + SC_STAGES) && ok; ++t) ok = load_tile(bh, t);
+          if (!ok || !mbar_wait(&bars[SB_CEMPTY], (sg - 1) & 1, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
         }
-        const uint32_t dst = sbase + L::KP_OFF + st * L::KTILE;
-        for (int r = rsub; r < 128; r += RSTEP) {
-          const int j = t * 128 + r;
-          const bool in = j < a.nK;
-          cp_async_16(dst + (u >> 3) * L::KCHUNK + sw128_off(r, u & 7),
-                      kp + (size_t)(in ? j : 0) * D + u * 8, in ? 16u : 0u);
-        }
-        mbar_arrive_cpasync(&bars[SB_FULL0 + st]);
+        mbar_arrive_expect_tx(&bars[SB_CFULL], L::CENT_BYTES);
+#pragma unroll
+        for (int ck = 0; ck < D / 64; ++ck)  // centroid rows qb0*8 .. qb0*8 + 255 of head bh
+          tma_load_3d(sbase + L::CENT_OFF + ck * L::CCHUNK, &tm_cent, ck * 64, qb0 * CMAX, bh, &bars[SB_CFULL]);
+        for (; t < t1 && ok; ++t) ok = load_tile(bh, t);
       }
+      // let copies still in flight land before the CTA can exit (only after an abort)
+      for (long long k = (it > SC_STAGES ? it - SC_STAGES : 0); k < it; ++k)
+        mbar_wait_quiet(&bars[SB_FULL0 + (int)(k % SC_STAGES)], (int)((k / SC_STAGES) & 1), timeout_ns);
+      if (sg > 0) mbar_wait_quiet(&bars[SB_CFULL], (sg - 1) & 1, timeout_ns);  // sg centroid loads issued
     }
-    cp_async_wait_all();
-  } else if (warp == 18) {
+    __syncwarp();
+  } else if (warp == SC_MMA_WARP) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC1 = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC2 = idesc_bf16_f32(128, SC_ROWS, 0, 0);
       long long it = 0;
       int sg = 0;
+      int nuse[2] = {0, 0};  // tiles issued into each TMEM buffer
       bool ok = true;
-      for (long long uu = u0; uu < u1 && ok; ++sg) {
-        long long unext, gi;
-        int k0, t0, t1;
-        segment(uu, unext, gi, k0, t0, t1);
-        uu = unext;
+      for (long long un = blockIdx.x; un < sp.U && ok; un += gridDim.x, ++sg) {
+        long long gi;
+        int t0, t1;
+        unit(un, gi, t0, t1);
         if (!(ok = mbar_wait(&bars[SB_CFULL], sg & 1, abort_flag, timeout_ns))) break;
         for (int t = t0; t < t1; ++t, ++it) {
-          const int st = (int)(it % SC_STAGES), b = (int)(it & 1);
+          const int st = (int)(it % SC_STAGES), b = (t - t0) & 1;
           ok = mbar_wait(&bars[SB_FULL0 + st], (int)((it / SC_STAGES) & 1), abort_flag, timeout_ns);
-          if (ok && it >= 2) ok = mbar_wait(&bars[SB_SFREE0 + b], (int)(((it >> 1) - 1) & 1), abort_flag, timeout_ns);
+          if (ok && nuse[b] > 0) ok = mbar_wait(&bars[SB_SFREE0 + b], (nuse[b] - 1) & 1, abort_flag, timeout_ns);
           if (!ok) break;
+          ++nuse[b];
           fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t cbase = sbase + L::CENT_OFF;
@@ -526,16 +547,15 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, Scor
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- consumers (warps 0-15)
-    const int q = warp & 3, sub = warp >> 2;
+    const int q = warp & 3, sub = (warp >> 2) & 1, grp = warp >> 3;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float c = a.scale_log2;
-    long long it = 0;
+    int nuse = 0;  // tiles of this group's TMEM buffer so far
     bool ok = true;
-    for (long long uu = u0; uu < u1;) {
-      long long unext, gi;
-      int k0, t0, t1;
-      segment(uu, unext, gi, k0, t0, t1);
-      uu = unext;
+    for (long long un = blockIdx.x; un < sp.U; un += gridDim.x) {
+      long long gi;
+      int t0, t1;
+      unit(un, gi, t0, t1);
       const long long bh = gi / sp.G;
       const int qb0 = (int)(gi - bh * sp.G) * SC_QB;
       if (PASS == 2) {
@@ -560,91 +580,92 @@ __global__ void __launch_bounds__(SC_THREADS, 1) score_kernel(SelectArgs a, Scor
         }
         asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
       }
-      const int h = sub >> 1, ch = sub & 1;  // pass 1: centroid half, key half
+      // pass 1: row sub * 128 + 32 q + lane (centroid half sub); pass 2: key 32 q + lane of the
+      // tile and centroid columns sub * 128 .. + 127 (query blocks sub * 16 .. + 15)
+      const uint32_t cols = (uint32_t)(sub * 128);
       float m = -INFINITY, z = 0.f;
-      for (int t = t0; t < t1; ++t, ++it) {
-        const int b = (int)(it & 1);
-        if (ok) ok = mbar_wait(&bars[SB_SFULL0 + b], (int)((it >> 1) & 1), abort_flag, timeout_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-          tc_fence_after();
-          if (PASS == 1) {
-            uint32_t v[64];
-            const uint32_t col = b * 256 + h * 128 + ch * 64;
-            tmem_ld_32x32b_x32(tmem + lane_off + col, *reinterpret_cast<uint32_t(*)[32]>(v));
-            tmem_ld_32x32b_x32(tmem + lane_off + col + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bars[SB_SFREE0 + b]);
-            const int jb = t * 128 + ch * 64;  // key of v[0]
-            if (jb + 64 > a.nK) {              // the ragged last tile: mask keys >= nK
+      auto compute = [&](uint32_t (&v)[32], int t, int part) {
+        if (PASS == 1) {
+          const int jb = t * 128 + part * 32;  // key of v[0]
+          if (jb + 32 > a.nK) {                // the ragged last tile: mask keys >= nK
 #pragma unroll
-              for (int k = 0; k < 64; ++k)
-                if (jb + k >= a.nK) v[k] = __float_as_uint(-INFINITY);
+            for (int e = 0; e < 32; ++e)
+              if (jb + e >= a.nK) v[e] = __float_as_uint(-INFINITY);
+          }
+          online_chunk(v, c, m, z);
+        } else {
+          const int j = t * 128 + q * 32 + lane;
+          const uint64_t c2 = f2_pack(c, c);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int cb = sub * 128 + part * 32 + qq * 8;  // first column of this query block
+            float mp[8];
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(mp[0]), "=f"(mp[1]), "=f"(mp[2]), "=f"(mp[3])
+                         : "r"(smem_u32(col_m + cb)));
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(mp[4]), "=f"(mp[5]), "=f"(mp[6]), "=f"(mp[7])
+                         : "r"(smem_u32(col_m + cb + 4)));
+            uint64_t acc = 0;  // (0.f, 0.f)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(v[qq * 8 + 2 * e]),
+                                                        __uint_as_float(v[qq * 8 + 2 * e + 1])),
+                                                c2, f2_pack(-mp[2 * e], -mp[2 * e + 1])));
+              acc = f2_add(acc, (e < SC_POLY_PAIRS2) ? exp2_poly_x2(x.x, x.y)
+                                                    : f2_pack(fast_exp2(x.x), fast_exp2(x.y)));
             }
-            online_chunk(v, c, m, z);
-            online_chunk(v + 32, c, m, z);
-          } else {
-            // two rounds of 32 columns (4 query blocks each); TMEM is released after the second
-            const int j = t * 128 + q * 32 + lane;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t v[32];
-              tmem_ld_32x32b_x32(tmem + lane_off + b * 256 + sub * 64 + half * 32, v);
-              tmem_wait_ld();
-              if (half == 1) {
-                tc_fence_before();
-                mbar_arrive(&bars[SB_SFREE0 + b]);
-              }
-#pragma unroll
-              for (int qq = 0; qq < 4; ++qq) {
-                const int cb = sub * 64 + half * 32 + qq * 8;  // first column of this query block
-                float mp[8];
-                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                             : "=f"(mp[0]), "=f"(mp[1]), "=f"(mp[2]), "=f"(mp[3])
-                             : "r"(smem_u32(col_m + cb)));
-                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                             : "=f"(mp[4]), "=f"(mp[5]), "=f"(mp[6]), "=f"(mp[7])
-                             : "r"(smem_u32(col_m + cb + 4)));
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                for (int k = 0; k < 8; k += 2) {
-                  s0 += fast_exp2(fmaf(__uint_as_float(v[qq * 8 + k]), c, -mp[k]));
-                  s1 += fast_exp2(fmaf(__uint_as_float(v[qq * 8 + k + 1]), c, -mp[k + 1]));
-                }
-                const int qb = qb0 + (cb >> 3);
-                if (j < a.nK && qb < a.nQ) a.S[((size_t)bh * a.nQ + qb) * a.nK + j] = s0 + s1;
-              }
-            }
+            const float2 sv = f2_unpack(acc);
+            const int qb = qb0 + (cb >> 3);
+            if (j < a.nK && qb < a.nQ) a.S[((size_t)bh * a.nQ + qb) * a.nK + j] = sv.x + sv.y;
           }
         }
-        if (PASS == 1 && (t + 1 == t1 || (t + 1) % sp.CT == 0)) {
-          // end of key chunk t / CT: merge the two key halves of each row into its slot.
-          // Each chunk's (m, z) depends only on its own keys, so S does not depend on how
-          // the units were dealt out to CTAs.
-          asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
-          const int row = h * 128 + q * 32 + lane;
-          if (ch == 1) merge[row] = make_float2(m, z);
-          asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
-          if (ch == 0 && ok) {
-            const float2 o = merge[row];
-            const float M = fmaxf(m, o.x);
-            float Z = 0.f;
-            if (M > -INFINITY) {
-              if (m > -INFINITY) Z += z * fast_exp2(m - M);
-              if (o.x > -INFINITY) Z += o.y * fast_exp2(o.x - M);
-            }
-            ((float2*)a.stats)[((size_t)gi * SC_ROWS + row) * SC_MAX_CHUNKS + t / sp.CT] = make_float2(M, Z);
+      };
+      // this group's tiles of the unit: t - t0 = grp, grp + 2, ... (they are in TMEM buffer
+      // grp), so the split, and with it the rounding of (m, z), depends only on the unit
+      for (int t = t0 + grp; t < t1; t += 2) {
+        if (ok) ok = mbar_wait(&bars[SB_SFULL0 + grp], nuse & 1, abort_flag, timeout_ns);
+        ++nuse;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) continue;
+        tc_fence_after();
+        const uint32_t base = tmem + lane_off + (uint32_t)(grp * 256) + cols;
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(base + part * 32, v);
+          tmem_wait_ld_regs(v);
+          if (part == 3) {  // the group has read its whole tile: the buffer is free
+            tc_fence_before();
+            mbar_arrive(&bars[SB_SFREE0 + grp]);
           }
-          m = -INFINITY;
-          z = 0.f;
+          compute(v, t, part);
+        }
+      }
+      if (PASS == 1) {
+        // merge the two groups' (m, z) of each row and store the unit's slot.  Each chunk's
+        // (m, z) depends only on its own keys, so S does not depend on how the units were
+        // dealt out to CTAs.
+        asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
+        const int row = sub * 128 + q * 32 + lane;
+        if (grp == 1) merge[row] = make_float2(m, z);
+        asm volatile("bar.sync 1, %0;" ::"n"(SC_CONSUMERS) : "memory");
+        if (grp == 0 && ok) {
+          const float2 o = merge[row];
+          const float M = fmaxf(m, o.x);
+          float Z = 0.f;
+          if (M > -INFINITY) {
+            if (m > -INFINITY) Z += z * fast_exp2(m - M);
+            if (o.x > -INFINITY) Z += o.y * fast_exp2(o.x - M);
+          }
+          ((float2*)a.stats)[((size_t)gi * SC_ROWS + row) * SC_MAX_CHUNKS + t0 / sp.CT] = make_float2(M, Z);
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 18) {
+  if (warp == SC_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
