@@ -39,6 +39,7 @@ constexpr int PLAN_SMEM_MAX_FLOATS = 40 * 1024;  // 160 KB of staged row (top-k 
 // 18,900 blocks staging wins (2.7 vs 3.6 ms).
 constexpr int PLAN_STAGE_MAX_FLOATS = 28 * 1024;
 constexpr uint64_t TWO32 = 1ull << 32;
+constexpr uint64_t kPlanTimeoutNs = 2000000000ull;  // bounded wait for the staged row
 
 struct PlanArgs {
   const float* S;   // [rows, nK] (not read in the uniform variant)
@@ -161,12 +162,92 @@ AB_DEV void block_exscan2_u64(uint64_t v0, uint64_t v1, uint64_t* red0, uint64_t
   total1 = t1;
 }
 
+// Block-wide sums of NU uint64 and ND double values with one barrier: each warp's lane 0
+// writes its partials into the slot set `par`, which alternates between calls, so a call
+// never overwrites slots that a thread may still be reading from the call before (every
+// thread has left that call's reads before it reaches this call's barrier).
+template <int NU, int ND>
+AB_DEV void block_sums(uint64_t (&u)[NU], double (&dv)[ND], uint64_t* ru, double* rd, int& par) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+#pragma unroll
+    for (int k = 0; k < NU; ++k) u[k] += __shfl_xor_sync(0xffffffffu, u[k], o);
+#pragma unroll
+    for (int k = 0; k < ND; ++k) dv[k] += __shfl_xor_sync(0xffffffffu, dv[k], o);
+  }
+  uint64_t* su = ru + par * 4 * PLAN_WARPS;
+  double* sd = rd + par * 2 * PLAN_WARPS;
+  if (l == 0) {
+#pragma unroll
+    for (int k = 0; k < NU; ++k) su[k * PLAN_WARPS + w] = u[k];
+#pragma unroll
+    for (int k = 0; k < ND; ++k) sd[k * PLAN_WARPS + w] = dv[k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < NU; ++k) {
+    uint64_t t = 0;
+#pragma unroll
+    for (int i = 0; i < PLAN_WARPS; ++i) t += su[k * PLAN_WARPS + i];
+    u[k] = t;
+  }
+#pragma unroll
+  for (int k = 0; k < ND; ++k) {
+    double t = 0.0;
+#pragma unroll
+    for (int i = 0; i < PLAN_WARPS; ++i) t += sd[k * PLAN_WARPS + i];
+    dv[k] = t;
+  }
+  par ^= 1;
+}
+
+// Exclusive scans in thread order of two uint64 values with one barrier (slot sets as above);
+// returns this thread's prefixes and the block totals.
+AB_DEV void block_exscan2_1b(uint64_t v0, uint64_t v1, uint64_t* ru, int& par, uint64_t& before0,
+                             uint64_t& before1, uint64_t& total0, uint64_t& total1) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  uint64_t inc0 = v0, inc1 = v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y0 = __shfl_up_sync(0xffffffffu, inc0, o);
+    const uint64_t y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+    if (l >= o) {
+      inc0 += y0;
+      inc1 += y1;
+    }
+  }
+  uint64_t* su = ru + par * 4 * PLAN_WARPS;
+  if (l == 31) {
+    su[w] = inc0;
+    su[PLAN_WARPS + w] = inc1;
+  }
+  __syncthreads();
+  uint64_t b0 = 0, b1 = 0, t0 = 0, t1 = 0;
+#pragma unroll
+  for (int i = 0; i < PLAN_WARPS; ++i) {
+    const uint64_t x0 = su[i], x1 = su[PLAN_WARPS + i];
+    if (i < w) {
+      b0 += x0;
+      b1 += x1;
+    }
+    t0 += x0;
+    t1 += x1;
+  }
+  before0 = b0 + inc0 - v0;
+  before1 = b1 + inc1 - v1;
+  total0 = t0;
+  total1 = t1;
+  par ^= 1;
+}
+
 template <bool STAGED>
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   extern __shared__ float srow_smem[];
-  __shared__ uint64_t red[PLAN_WARPS];
-  __shared__ uint64_t red2[PLAN_WARPS];
-  __shared__ double redd[PLAN_WARPS];
+  __shared__ uint64_t ru[2 * 4 * PLAN_WARPS];
+  __shared__ double rd[2 * 2 * PLAN_WARPS];
+  __shared__ uint64_t row_bar;  // bulk staging of the row
+  int par = 0;  // reduction slot set
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nK = a.nK;
@@ -210,7 +291,34 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         ++npos;
       }
     };
-    if (STAGED) {
+    const bool bulk = STAGED && !uniform && ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
+    if (bulk) {
+      // the whole row in one bulk copy (one request in flight instead of a dependent
+      // chain of loads per thread), then the sums over this thread's chunk
+      if (tid == 0) {
+        mbar_init(&row_bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&row_bar, (uint32_t)nK * 4u);
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                smem_u32(srow_smem)),
+            "l"(grow), "r"((uint32_t)nK * 4u), "r"(smem_u32(&row_bar))
+            : "memory");
+      }
+      __syncthreads();  // the barrier is initialised before anyone waits on it
+      const bool landed = mbar_wait_quiet(&row_bar, 0, kPlanTimeoutNs);
+      if (__syncthreads_or(!landed)) {
+        if (tid == 0) ab_flag(AB_ERR_DEVICE_TIMEOUT);
+        return;
+      }
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = reinterpret_cast<const float4*>(srow_smem)[i];
+        acc(v.x);
+        acc(v.y);
+        acc(v.z);
+        acc(v.w);
+      }
+    } else if (STAGED) {
       const bool vec = ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
       float4* s4 = reinterpret_cast<float4*>(srow_smem);
       for (int j = tid; j < nK4; j += PLAN_THREADS) {
@@ -234,7 +342,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         acc(v.z);
         acc(v.w);
       }
-      // read by other threads only after the barriers of the block sum below
+      // read by other threads only after the barrier of the block sum below
     } else {
       for (int i = c0; i < c1; ++i) {
         const float4 v = load4(i);
@@ -246,123 +354,166 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     }
     tot = (double)sum - (double)comp;
   }
-  block_sum_cd(npos, tot, red, redd);
+  {
+    uint64_t u1[1] = {npos};
+    double d1[1] = {tot};
+    block_sums<1, 1>(u1, d1, ru, rd, par);
+    npos = u1[0];
+    tot = d1[0];
+  }
   const bool reachable = npos >= s;
 
   // ---- lambda*: the smallest positive fp32 (bit pattern in (0, 0x7F800000]) with
-  // F(lambda) >= s 2^32.  F is monotone in the bit pattern, so any search that brackets
-  // the boundary and bisects finds the same lambda as a full 31-step bisection.
-  // F(bits) also leaves this thread's part -- its saturated count and the sum of its other
-  // q_j -- in (ev_nsat, ev_q), and with `want_rest` the block sum of the unsaturated scores.
-  uint32_t ev_nsat = 0;
-  uint64_t ev_q = 0;
-  auto F = [&](uint32_t bits, bool want_rest, double* rest_out) -> uint64_t {
-    const float lam = __uint_as_float(bits);
-    uint32_t ns = 0;
-    uint64_t qs = 0;
+  // F(lambda) >= s 2^32.  F is monotone in the bit pattern, so any search that brackets the
+  // boundary between lo (F < target, or lo = 0) and hi (F >= target, or hi = +inf, where
+  // F = |positive| 2^32 >= target) and bisects finds the same lambda as a full 31-step
+  // bisection.  An evaluation also leaves this thread's part of F -- its saturated count and
+  // the sum of its other q_j -- which the output needs at lambda*.
+  //
+  // First pass: F at the three fp32 neighbours b0 - 1, b0, b0 + 1 of lambda0 = s / sum(S)
+  // (and the sum of the scores unsaturated at b0).  Without saturation F(lambda) is
+  // 2^32 lambda sum(S) less the truncations (under nK units, far below the 2^32 lambda ulp
+  // sum(S) that one fp32 step adds), so lambda* is b0 or b0 + 1 and this one pass brackets it.
+  uint32_t lo = 0u, hi = 0x7F800000u;
+  bool hi_known = false;  // whether (hi_nsat, hi_q) hold this thread's part of F(hi)
+  uint32_t hi_nsat = 0;
+  uint64_t hi_q = 0;
+  if (reachable) {
+    const float lam0 = (tot > 0.0) ? (float)((double)a.s / tot) : 0.f;
+    uint32_t b0 = __float_as_uint(lam0);
+    if (!(lam0 > 0.f) || !isfinite(lam0)) b0 = 0x3F800000u;  // 1.0: any start works
+    b0 = min(max(b0, 2u), 0x7F7FFFFEu);                       // three finite positive neighbours
+    const float l3[3] = {__uint_as_float(b0 - 1u), __uint_as_float(b0), __uint_as_float(b0 + 1u)};
+    uint32_t ns[3] = {0u, 0u, 0u};
+    uint64_t qs[3] = {0ull, 0ull, 0ull};
     float rest = 0.f;
     for (int i = c0; i < c1; ++i) {
       const float4 v = load4(i);
       const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        uint32_t q;
-        const bool sat = fixed_q32(lam, x4[k], q);
-        ns += sat;
-        qs += sat ? 0u : q;
-        if (want_rest && !sat && x4[k] > 0.f) rest += x4[k];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          uint32_t q;
+          const bool sat = fixed_q32(l3[c], x4[k], q);  // q = 0 when saturated
+          ns[c] += sat;
+          qs[c] += q;
+          if (c == 1 && !sat && x4[k] > 0.f) rest += x4[k];
+        }
       }
     }
-    ev_nsat = ns;
-    ev_q = qs;
-    uint64_t part = ((uint64_t)ns << 32) + qs;  // per thread below 2^39
-    if (want_rest) {
-      double r = rest;
-      block_sum_cd(part, r, red, redd);
-      *rest_out = r;
-      return part;
-    }
-    return block_sum_u64(part, red);
-  };
-  uint32_t lo = 0u, hi = 0x7F800000u;
-  bool hi_known = false;  // whether (hi_nsat, hi_q) hold this thread's part of F(hi)
-  uint32_t hi_nsat = 0;
-  uint64_t hi_q = 0;
-  auto take_hi = [&](uint32_t bits) {
-    hi = bits;
-    hi_nsat = ev_nsat;
-    hi_q = ev_q;
-    hi_known = true;
-  };
-  if (reachable) {
-    // Start at lambda0 = s / sum(S) and take one Newton step on the exact integer sum:
-    // F grows by about (sum of the unsaturated scores) * 2^32 per unit lambda, so the step
-    // is the water-filling update lambda <- (s - |saturated|) / (unsaturated sum).  On
-    // typical rows the two points bracket lambda* to one ulp.
-    const float lam0 = (tot > 0.0) ? (float)((double)a.s / tot) : 0.f;
-    uint32_t b = __float_as_uint(lam0);
-    if (!(lam0 > 0.f) || !isfinite(lam0)) b = 0x3F800000u;  // 1.0: any start works
-    double rest = 0.0;
-    uint64_t fb = F(b, true, &rest);
-    uint32_t b_nsat = ev_nsat;
-    uint64_t b_q = ev_q;
-    auto point_b_is_hi = [&]() {
-      hi = b;
-      hi_nsat = b_nsat;
-      hi_q = b_q;
+    uint64_t f3[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) f3[c] = ((uint64_t)ns[c] << 32) + qs[c];  // per thread below 2^39
+    double r1[1] = {(double)rest};
+    block_sums<3, 1>(f3, r1, ru, rd, par);
+    // F is monotone: lo / hi from the three points
+    int kstar = 3;  // first candidate with F >= target
+#pragma unroll
+    for (int c = 2; c >= 0; --c)
+      if (f3[c] >= target) kstar = c;
+    if (kstar < 3) {
+      hi = b0 - 1u + (uint32_t)kstar;
+      hi_nsat = kstar == 0 ? ns[0] : (kstar == 1 ? ns[1] : ns[2]);  // kstar is block-uniform
+      hi_q = kstar == 0 ? qs[0] : (kstar == 1 ? qs[1] : qs[2]);
       hi_known = true;
-    };
-    if (rest > 0.0) {
-      const double lam_n = (double)__uint_as_float(b) +
-                           ((double)target - (double)fb) / (rest * 4294967296.0);
+    }
+    bool lo_set = kstar > 0;  // F(lo) < target was evaluated (else lo = 0, F(0) = 0)
+    if (lo_set) lo = b0 - 2u + (uint32_t)kstar;
+    if (hi - lo > 1u && r1[0] > 0.0) {
+      // Newton on the exact integer sum from b0: F grows by about (sum of the unsaturated
+      // scores) 2^32 per unit lambda (the water-filling update).
+      const double lam_n = (double)l3[1] + ((double)target - (double)f3[1]) / (r1[0] * 4294967296.0);
       const float lf = (float)lam_n;
-      if (lf > 0.f && isfinite(lf) && __float_as_uint(lf) != b) {
-        const uint32_t b2 = __float_as_uint(lf);
-        const uint64_t f2 = F(b2, false, nullptr);
-        if ((f2 >= target) == (fb >= target)) {  // same side: continue from the Newton point
-          b = b2;
-          fb = f2;
-          b_nsat = ev_nsat;
-          b_q = ev_q;
-        } else if (b2 > b) {
-          lo = b;
-          take_hi(b2);
+      const uint32_t b2 = __float_as_uint(lf);
+      if (lf > 0.f && isfinite(lf) && b2 > lo && b2 < hi) {
+        uint64_t f1[1];
+        uint32_t ns2 = 0;
+        uint64_t qs2 = 0;
+        for (int i = c0; i < c1; ++i) {
+          const float4 v = load4(i);
+          const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t q;
+            ns2 += fixed_q32(lf, x4[k], q);
+            qs2 += q;
+          }
+        }
+        f1[0] = ((uint64_t)ns2 << 32) + qs2;
+        double none[1] = {0.0};
+        block_sums<1, 1>(f1, none, ru, rd, par);
+        if (f1[0] >= target) {
+          hi = b2;
+          hi_nsat = ns2;
+          hi_q = qs2;
+          hi_known = true;
         } else {
           lo = b2;
-          point_b_is_hi();
+          lo_set = true;
         }
       }
     }
-    const bool bracketed = !(lo == 0u && hi == 0x7F800000u);  // by the Newton point
-    if (!bracketed) {
-      if (fb >= target) {  // boundary at or below b: step down
-        point_b_is_hi();
-        uint32_t step = 1;
-        while (true) {
-          const uint32_t cand = (hi > step) ? hi - step : 0u;
-          if (cand == 0u || F(cand, false, nullptr) < target) { lo = cand; break; }
-          take_hi(cand);
-          step <<= 1;
-        }
-      } else {  // boundary above b: step up
-        lo = b;
-        uint32_t step = 1;
-        while (true) {
-          const uint32_t cand = (0x7F800000u - lo > step) ? lo + step : 0x7F800000u;
-          if (cand == 0x7F800000u) { hi = cand; hi_known = false; break; }
-          if (F(cand, false, nullptr) >= target) { take_hi(cand); break; }
-          lo = cand;
-          step <<= 1;
-        }
-      }
-    }
+    // the rest (rare): doubling steps away from the evaluated side until the other side is
+    // evaluated too (lambda = +inf and lambda = 0 are the outer bounds), then bisection
+    uint32_t step = 1;
     while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (F(mid, false, nullptr) >= target) take_hi(mid); else lo = mid;
+      uint32_t cand;
+      if (!hi_known) {  // step up from lo
+        cand = (0x7F800000u - lo > step) ? lo + step : 0x7F800000u;
+        step <<= 1;
+      } else if (!lo_set) {  // step down from hi
+        if (hi <= step) {    // reached lambda = 0: bisect [0, hi]
+          lo = 0u;
+          lo_set = true;
+          continue;
+        }
+        cand = hi - step;
+        step <<= 1;
+      } else {
+        cand = lo + ((hi - lo) >> 1);
+      }
+      uint32_t ns2 = 0;
+      uint64_t qs2 = 0;
+      const float lc = __uint_as_float(cand);
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t q;
+          ns2 += fixed_q32(lc, x4[k], q);
+          qs2 += q;
+        }
+      }
+      uint64_t f1[1] = {((uint64_t)ns2 << 32) + qs2};
+      double none[1] = {0.0};
+      block_sums<1, 1>(f1, none, ru, rd, par);
+      if (f1[0] >= target) {
+        hi = cand;
+        hi_nsat = ns2;
+        hi_q = qs2;
+        hi_known = true;
+      } else {
+        lo = cand;
+        lo_set = true;
+      }
     }
-    if (!hi_known) {  // lambda* = +inf was never evaluated (pathological rows)
-      F(hi, false, nullptr);
-      take_hi(hi);
+    if (!hi_known) {  // lambda* = +inf (pathological rows): its part of F
+      uint32_t ns2 = 0;
+      uint64_t qs2 = 0;
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t q;
+          ns2 += fixed_q32(__uint_as_float(hi), x4[k], q);
+          qs2 += q;
+        }
+      }
+      hi_nsat = ns2;
+      hi_q = qs2;
     }
   }
   const float lam = __uint_as_float(hi);
@@ -388,7 +539,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     }
   }
   uint64_t sat_before, rest_before, n_sat, tot_rest;
-  block_exscan2_u64(my_sat, my_rest, red, red2, sat_before, rest_before, n_sat, tot_rest);
+  block_exscan2_1b(my_sat, my_rest, ru, par, sat_before, rest_before, n_sat, tot_rest);
 
   const uint32_t U = philox4x32_10_w0((uint32_t)(a.row0 + row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
                                       0u, (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
@@ -398,14 +549,17 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   // Saturated blocks come first in the layout, block k of them covering [k 2^32, (k+1) 2^32):
   // each holds exactly one lattice point, so every saturated block is drawn.  The other
   // blocks follow in ascending order; this thread's chunk covers [start, start + my_rest).
-  // With the budget unreachable, the first s - n_sat zero blocks (in order) complete it.
+  // The intervals of the threads before this one are contiguous, so the draws before this
+  // thread's first output are its predecessors' saturated blocks plus the lattice points in
+  // [n_sat 2^32, start).  With the budget unreachable, the first s - n_sat zero blocks (in
+  // order) complete the draw.
   const uint64_t start = n_sat * TWO32 + rest_before;
   const uint64_t need = s - min(n_sat, s);
-  const uint64_t my_sel =
-      my_sat + (reachable ? below(min(start + my_rest, target)) - below(min(start, target))
-                          : (rest_before < need ? min(my_rest, need - rest_before) : 0ull));
-  uint64_t out_before, zero_b, n_sel, zero_t;
-  block_exscan2_u64(my_sel, 0ull, red, red2, out_before, zero_b, n_sel, zero_t);
+  const uint64_t base = n_sat * TWO32;
+  const uint64_t out_before =
+      sat_before + (reachable ? below(min(start, target)) - below(min(base, target)) : min(rest_before, need));
+  const uint64_t n_sel =
+      n_sat + (reachable ? below(min(base + tot_rest, target)) - below(min(base, target)) : min(tot_rest, need));
   if (n_sel != s && tid == 0) ab_flag(AB_ERR_DEVICE_CHECK);  // cannot happen; guards the writes
 
   // ---- write ascending idx and the fixed-point probability (its log follows below)
@@ -461,11 +615,22 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   {
     float* olp = a.logpi + (size_t)row * a.s;
     uint32_t* raw = reinterpret_cast<uint32_t*>(olp);
-    for (int o = tid; o < a.s; o += PLAN_THREADS) {
-      const uint32_t q = raw[o];
-      olp[o] = (q == 0xFFFFFFFFu || a.mode == AB_PLAN_SIP_NO_IPW)
-                   ? 0.f
-                   : (float)log((double)q * (1.0 / 4294967296.0));
+    constexpr int LB = 4;  // outputs per batch: their loads are in flight together
+    for (int o0 = tid; o0 < a.s; o0 += LB * PLAN_THREADS) {
+      uint32_t q[LB];
+#pragma unroll
+      for (int k = 0; k < LB; ++k) {
+        const int o = o0 + k * PLAN_THREADS;
+        q[k] = o < a.s ? raw[o] : 0xFFFFFFFFu;
+      }
+#pragma unroll
+      for (int k = 0; k < LB; ++k) {
+        const int o = o0 + k * PLAN_THREADS;
+        if (o < a.s)
+          olp[o] = (q[k] == 0xFFFFFFFFu || a.mode == AB_PLAN_SIP_NO_IPW)
+                       ? 0.f
+                       : (float)log((double)q[k] * (1.0 / 4294967296.0));
+      }
     }
   }
 }
