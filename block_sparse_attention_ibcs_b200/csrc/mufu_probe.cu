@@ -1,9 +1,11 @@
-// Exponential throughput probe (a stand-alone executable, not part of the library).
+// Throughput probe (a stand-alone executable, not part of the library).
 //
-// Measures exp2 results per SM per clock on the MUFU (ex2.approx) and on the FMA pipe
-// (the packed-pair polynomial the selector uses for part of its exponentials), with
-// 148 CTAs of W warps each running ILP independent chains; only a per-CTA clock count and
-// one float per thread are written.  Used to set the selector's exponential bound.
+// Measures, per SM per clock: exp2 results on the MUFU (ex2.approx) and on the FMA pipe
+// (the packed-pair polynomial the selector uses for part of its exponentials); and fp64
+// additions of bf16 values widened to double (by conversion, or built from the bits with
+// integer operations), the inner step of the selector's exact means.  148 CTAs of W warps
+// each run independent chains; only a per-CTA clock count and one value per thread are
+// written.
 #include <cstdio>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -49,6 +51,45 @@ void run(int warps, float* out, long long* cyc) {
          (double)warps * 32 * iters * ILP / mx);
 }
 
+template <int MODE>
+__global__ void f64_probe(const uint32_t* in, double* out, int iters, long long* cyc) {
+  uint32_t w[8];
+  for (int i = 0; i < 8; ++i) w[i] = in[(threadIdx.x + i * 37) & 1023] | 0x3f803f80u;
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const long long t0 = clock64();
+  for (int n = 0; n < iters; ++n) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t x = w[i] + n;  // upper half: a normal bf16
+      double d;
+      if (MODE == 0) {
+        d = (double)__uint_as_float(x & 0xffff0000u);
+      } else {  // sign | (exponent + 1023 - 127, mantissa) in the high word
+        d = __hiloint2double((int)((((x >> 3) & 0x0FFFE000u) + 0x38000000u) | (x & 0x80000000u)), 0);
+      }
+      acc[i] += d;
+    }
+  }
+  const long long t1 = clock64();
+  double s = 0.0;
+  for (int i = 0; i < 8; ++i) s += acc[i];
+  out[blockIdx.x * blockDim.x + threadIdx.x] = s;
+  if (threadIdx.x == 0) cyc[blockIdx.x] = t1 - t0;
+}
+
+template <int MODE>
+void run_f64(int warps, const uint32_t* in, double* out, long long* cyc) {
+  const int iters = 1000;
+  for (int rep = 0; rep < 2; ++rep) f64_probe<MODE><<<148, warps * 32>>>(in, out, iters, cyc);
+  cudaDeviceSynchronize();
+  long long h[148];
+  cudaMemcpy(h, cyc, sizeof(h), cudaMemcpyDeviceToHost);
+  double mx = 0;
+  for (int i = 0; i < 148; ++i) mx = h[i] > mx ? (double)h[i] : mx;
+  printf("fp64 add of bf16 (%s) warps/SM=%2d: %.2f per clock per SM\n", MODE ? "built from bits" : "converted",
+         warps, (double)warps * 32 * iters * 8 / mx);
+}
+
 int main() {
   float* out;
   long long* cyc;
@@ -56,6 +97,12 @@ int main() {
   cudaMalloc(&cyc, 148 * 8);
   for (int w : {4, 8, 16, 32}) { run<0, 8>(w, out, cyc); run<0, 16>(w, out, cyc); }
   for (int w : {4, 8, 16, 32}) { run<1, 8>(w, out, cyc); run<1, 16>(w, out, cyc); }
+  uint32_t* in;
+  double* out64;
+  cudaMalloc(&in, 1024 * 4);
+  cudaMemset(in, 0, 1024 * 4);
+  cudaMalloc(&out64, 148 * 1024 * 8);
+  for (int w : {8, 16, 32}) { run_f64<0>(w, in, out64, cyc); run_f64<1>(w, in, out64, cyc); }
   const cudaError_t e = cudaGetLastError();
   printf("status: %s\n", cudaGetErrorString(e));
   return e == cudaSuccess ? 0 : 1;

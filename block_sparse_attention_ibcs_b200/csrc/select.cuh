@@ -56,21 +56,34 @@ __global__ void pool_kernel(SelectArgs a) {
     const int t0 = j * a.bk, t1 = min(a.N, t0 + a.bk);
     double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const uint16_t* src = a.K + (bh * a.N + t0) * D + u * 8;
-    for (int t = t0; t < t1; ++t, src += D) {
-      const uint4 v = __ldg((const uint4*)src);
+    auto add_row = [&](const uint4 v) {
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         acc[2 * e] += bf16_to_double((uint16_t)(w4[e] & 0xffffu));
         acc[2 * e + 1] += bf16_to_double((uint16_t)(w4[e] >> 16));
       }
+    };
+    const int n = t1 - t0;
+    if (n == 4) {  // the usual 4-token block: its four row loads in flight together
+      uint4 v[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) v[t] = __ldg((const uint4*)(src + t * D));
+#pragma unroll
+      for (int t = 0; t < 4; ++t) add_row(v[t]);
+    } else {
+      for (int t = 0; t < n; ++t) add_row(__ldg((const uint4*)(src + t * D)));
     }
-    const double cnt = (double)(t1 - t0);
+    // a power-of-two count divides exactly as a multiplication by its reciprocal
+    const double cnt = (double)n, inv = 1.0 / cnt;
+    const bool pow2 = (n & (n - 1)) == 0;
     uint32_t o[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      o[e] = (uint32_t)bf16_bits_from_double(acc[2 * e] / cnt) |
-             ((uint32_t)bf16_bits_from_double(acc[2 * e + 1] / cnt) << 16);
+    for (int e = 0; e < 4; ++e) {
+      const double m0 = pow2 ? acc[2 * e] * inv : acc[2 * e] / cnt;
+      const double m1 = pow2 ? acc[2 * e + 1] * inv : acc[2 * e + 1] / cnt;
+      o[e] = (uint32_t)bf16_bits_from_double(m0) | ((uint32_t)bf16_bits_from_double(m1) << 16);
+    }
     *(uint4*)(a.Kp + bj * D + u * 8) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
@@ -79,9 +92,11 @@ __global__ void pool_kernel(SelectArgs a) {
 //
 // One CTA of 256 threads per (bh, query block).
 //  * Segment means (the start) and member means (the update) are exact fp64 sums of the
-//    bf16 rows divided by the count (IEEE division), as the CPU reference computes them.
-//    The update visits the rows in label order (a counting sort), so each thread (one
-//    dimension) runs through the rows once, accumulating into the current cluster.
+//    bf16 rows divided by the count (IEEE division; a power-of-two count as the exact
+//    multiplication by its reciprocal), as the CPU reference computes them.  Sums of at
+//    most 128 bf16 values are exact in fp64, so their order does not matter: the update
+//    visits the rows in label order (a counting sort), two or four threads per dimension
+//    taking alternate rows of each cluster and adding their partial sums by shuffles.
 //  * Assignment: two threads per row compute the 8 squared distances in fp32 against the
 //    fp32-rounded centroids.  With u = 2^-24 and n = d terms, the fp32 distance differs
 //    from the exact one by at most (n + 4) u (2 |q|^2 + 2 |c|^2) (rounding of c, of q - c,
@@ -131,7 +146,8 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
     if (c < C) {
       const int s0 = c * n / C, s1 = (c + 1) * n / C;
       for (int r = s0; r < s1; ++r) acc += bf16_to_double(qs[r * D + dd]);
-      if (s1 > s0) acc = acc / (double)(s1 - s0);
+      const int len = s1 - s0;
+      if (len > 0) acc = ((len & (len - 1)) == 0) ? acc * (1.0 / (double)len) : acc / (double)len;
     }
     c64[p] = acc;
   }
@@ -243,15 +259,20 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
     __syncthreads();
     if (tid < n) perm[atomicAdd(&off[lab[tid]], 1)] = (uint8_t)tid;  // off[c] ends at its cluster's end
     __syncthreads();
-    // update: each thread owns a dimension and walks the rows grouped by cluster
-    if (tid < D) {
+    // update: KM_THREADS / D adjacent threads share a dimension and walk alternate rows of
+    // each cluster (label order); their partial sums meet by shuffles
+    {
+      constexpr int PARTS = KM_THREADS / D;  // 2 at d = 128, 4 at d = 64
+      const int dd = tid / PARTS, h = tid % PARTS;
       int r0 = 0;
       for (int c = 0; c < CMAX; ++c) {
-        const int k = cnt[c];
+        const int k = cnt[c];  // block-uniform
         if (k > 0) {
           double acc = 0.0;
-          for (int q = r0; q < r0 + k; ++q) acc += bf16_to_double(qs[perm[q] * D + tid]);
-          c64[c * D + tid] = acc / (double)k;
+          for (int q = r0 + h; q < r0 + k; q += PARTS) acc += bf16_to_double(qs[perm[q] * D + dd]);
+#pragma unroll
+          for (int o = 1; o < PARTS; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (h == 0) c64[c * D + dd] = acc / (double)k;
         }
         r0 += k;
       }
