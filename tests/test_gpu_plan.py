@@ -125,3 +125,42 @@ def test_sample_monte_carlo_inclusion_frequencies():
     se = np.sqrt(np.maximum(pi * (1 - pi), 1e-12) / R)
     assert np.abs((hits - pi) / se)[(pi > 0) & (pi < 1)].max() < 5.5
     assert (hits[pi == 1] == 1).all()
+
+
+def test_plan_stress_rows_every_path():
+    """Many varied rows, every one bit-exact.  Of the 8,000 (row, s) cases the planner's
+    search brackets lambda* in its single three-candidate pass for 3,837, after the Newton
+    step for 447, after doubling and bisection for 2,708, and 1,008 have fewer positive
+    scores than s (counted by a CPU emulation of the search).  The step down from below the
+    three candidates needs every product at lambda0's lower neighbour rounded up by the
+    full 2^-24, which these rows never reach."""
+    rng = np.random.default_rng(12)
+    nK, R = 256, 2000
+    rows = []
+    for r in range(R):
+        kind = r % 8
+        if kind == 0:
+            x = rng.dirichlet(np.full(nK, 0.05))                           # very peaked
+        elif kind == 1:
+            x = np.exp(rng.uniform(0.5, 8.0) * rng.standard_normal(nK))    # heavy tails
+        elif kind == 2:
+            x = rng.dirichlet(np.full(nK, 1.0)) * 10.0 ** rng.uniform(-6, 6)  # unnormalised
+        elif kind == 3:
+            x = np.full(nK, 1.0 / nK) * (1 + 1e-7 * rng.standard_normal(nK))  # near ties
+        elif kind == 4:
+            x = rng.dirichlet(np.full(nK, 0.3)); x[rng.random(nK) < 0.7] = 0.0  # many zeros
+        elif kind == 5:
+            x = np.zeros(nK); x[rng.integers(0, nK, 3)] = rng.random(3) + 0.1   # few positive
+        elif kind == 6:
+            x = rng.dirichlet(np.full(nK, 0.5)); x[rng.integers(0, nK, 2)] = np.nan
+            x[rng.integers(0, nK, 2)] = -1.0                                 # NaN / negative
+        else:
+            x = rng.random(nK) ** 12                                         # skewed uniform
+        rows.append(x)
+    S = np.stack(rows).astype(np.float32)
+    # one launch covers B*H*nQ rows: R/8 heads of 8 query blocks (N = 1024, nK = 256)
+    p = ab.params(1, R // 8, 1024, 64, kv_block=4)
+    St = torch.from_numpy(S).cuda().reshape(1, R // 8, 8, nK)
+    for s in (1, 7, 64, 200):
+        idx, lp = _gpu_plan(p, St, s, 77, 5)
+        _check_rows(S, idx, lp, s, 77, 5, range(R))
