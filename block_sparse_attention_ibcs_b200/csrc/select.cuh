@@ -98,11 +98,14 @@ __global__ void pool_kernel(SelectArgs a) {
 //    visits the rows in label order (a counting sort), two or four threads per dimension
 //    taking alternate rows of each cluster and adding their partial sums by shuffles.
 //  * Assignment: two threads per row compute the 8 squared distances in fp32 against the
-//    fp32-rounded centroids.  With u = 2^-24 and n = d terms, the fp32 distance differs
-//    from the exact one by at most (n + 4) u (2 |q|^2 + 2 |c|^2) (rounding of c, of q - c,
-//    and of the n-term sum), so when the best and second-best fp32 distances are further
-//    apart than the sum of their bounds the fp32 choice is the exact argmin.  Rows inside
-//    the margin are recomputed in fp64 (ties to the lowest cluster), like the reference.
+//    fp32-rounded centroids as |q|^2 + |c|^2 - 2 q.c (one fma per column and centroid).
+//    With u = 2^-24 each fp32 distance is within (d + d/32 + 14) u (|q|^2 + |c|^2) of the
+//    exact one: the two d/2-term q.c chains and their sum (doubled), the rounding of c to
+//    fp32, the |q|^2 and |c|^2 sums, and the final two roundings (|q.c| is at most half of
+//    |q|^2 + |c|^2).  So when the best and second-best fp32 distances are further apart
+//    than the best's bound plus the largest bound of any cluster, the fp32 choice is the
+//    exact argmin.  Rows inside the margin are recomputed in fp64 (ties to the lowest
+//    cluster), like the reference.
 
 template <int D>
 __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
@@ -190,36 +193,38 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) q2 = fmaf(qv[k], qv[k], q2);
 #pragma unroll
-        for (int c = 0; c < CMAX; ++c) {
+        for (int c = 0; c < CMAX; ++c) {  // dist[c] accumulates q . c here
           const float* cc = cf + c * D + ah * H + e;
           const float4 c0 = *(const float4*)cc;
           const float4 c1 = *(const float4*)(cc + 4);
-          const float dv[8] = {qv[0] - c0.x, qv[1] - c0.y, qv[2] - c0.z, qv[3] - c0.w,
-                               qv[4] - c1.x, qv[5] - c1.y, qv[6] - c1.z, qv[7] - c1.w};
+          const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-          for (int k = 0; k < 8; ++k) dist[c] = fmaf(dv[k], dv[k], dist[c]);
+          for (int k = 0; k < 8; ++k) dist[c] = fmaf(qv[k], cv[k], dist[c]);
         }
       }
 #pragma unroll
       for (int c = 0; c < CMAX; ++c) dist[c] += __shfl_xor_sync(0xffffffffu, dist[c], 1);
       q2 += __shfl_xor_sync(0xffffffffu, q2, 1);
+#pragma unroll
+      for (int c = 0; c < CMAX; ++c) dist[c] = (q2 + c2[c]) - 2.f * dist[c];  // |q - c|^2
       int best = -1, second = -1;
-      float d1 = 0.f, d2 = 0.f, n1 = 0.f, n2 = 0.f;  // best / second distance and |c|^2
+      float d1 = 0.f, d2 = 0.f, n1 = 0.f, nmax = 0.f;  // best / second distance, |c_best|^2, max |c|^2
 #pragma unroll
       for (int c = 0; c < CMAX; ++c) {
         if (!alive[c]) continue;
+        nmax = fmaxf(nmax, c2[c]);
         if (best < 0 || dist[c] < d1) {
-          second = best; d2 = d1; n2 = n1;
+          second = best; d2 = d1;
           best = c; d1 = dist[c]; n1 = c2[c];
         } else if (second < 0 || dist[c] < d2) {
-          second = c; d2 = dist[c]; n2 = c2[c];
+          second = c; d2 = dist[c];
         }
       }
       constexpr float U = 5.9604645e-8f;  // 2^-24
       bool certain = true;
       if (second >= 0) {
-        const float kb = (float)(D + 4) * U * 2.f * 1.0625f;  // bound factor with margin
-        certain = d2 - d1 > kb * ((q2 + n1) + (q2 + n2));
+        const float kb = (float)(D + D / 32 + 16) * U * 1.0625f;  // bound factor with margin
+        certain = d2 - d1 > kb * ((q2 + n1) + (q2 + nmax));
       }
       // rows whose fp32 margin is too small: recompute all distances in fp64
       if (__any_sync(0xffffffffu, !certain && ar < n)) {
