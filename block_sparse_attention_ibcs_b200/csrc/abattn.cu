@@ -116,9 +116,11 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// split_bh: the head count the score passes' work split is chosen for (the whole tensor's,
+// also when this launch covers a slice of its heads)
 template <int D>
 ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, const Workspace& ws,
-                     int8_t* labels, cudaStream_t st) {
+                     int8_t* labels, cudaStream_t st, long long split_bh = 0) {
   SelectArgs a;
   a.Q = (const uint16_t*)Q;
   a.K = (const uint16_t*)K;
@@ -140,7 +142,7 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
   const int pool_blocks = (int)((units + 255) / 256 < 148 * 32 ? (units + 255) / 256 : 148 * 32);
   pool_kernel<D><<<pool_blocks, 256, 0, st>>>(a);
   kmeans_kernel<D><<<(unsigned)(d.BH * d.nQ), KM_THREADS, 0, st>>>(a);
-  const ScoreSplit sp = score_split(d.BH, d.nQ, d.nK);
+  const ScoreSplit sp = score_split(d.BH, d.nQ, d.nK, split_bh > 0 ? split_bh : d.BH);
   using SL = ScoreSmem<D>;
   if (cudaFuncSetAttribute(score_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SL::ALLOC) != cudaSuccess ||
@@ -314,8 +316,8 @@ ab_status select_plan_slice(const Dims& d, long long bh0, long long n, const voi
   const void* Kg = (const uint16_t*)K + qk;
   float* Sg = S + (size_t)bh0 * d.nQ * d.nK;
   Workspace wsp = carve(g, ws);
-  ab_status r = (d.d == 128) ? run_select<128>(g, Qg, Kg, Sg, wsp, nullptr, st_sel)
-                             : run_select<64>(g, Qg, Kg, Sg, wsp, nullptr, st_sel);
+  ab_status r = (d.d == 128) ? run_select<128>(g, Qg, Kg, Sg, wsp, nullptr, st_sel, d.BH)
+                             : run_select<64>(g, Qg, Kg, Sg, wsp, nullptr, st_sel, d.BH);
   if (r != AB_OK) return r;
   if (st_plan != st_sel) {
     if (cudaEventRecord(ev, st_sel) != cudaSuccess || cudaStreamWaitEvent(st_plan, ev, 0) != cudaSuccess)

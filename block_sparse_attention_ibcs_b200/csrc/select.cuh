@@ -301,8 +301,8 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
 //
 // The page's batched scoring ("premises & limits": query/KV blocks scored as batched
 // matrix operations) as two persistent tensor-core streaming passes.  A group is 32 query
-// blocks of one head (256 centroid rows); its key axis is cut into chunks of whole
-// 128-key tiles.  The (group, chunk) units, numbered head by head, are dealt out
+// blocks of one head (256 centroid rows); its key axis is cut into at most 8 chunks of
+// whole 128-key tiles (the count chosen per shape, see score_split).  The (group, chunk) units, numbered head by head, are dealt out
 // round-robin to one CTA per SM, so the CTAs running at any moment work on about one
 // head and share its pooled keys in L2 (all heads' pooled keys together exceed L2 at the
 // Wan2.1-14B shape).  A CTA loads a unit's centroids, then streams the chunk's key tiles;
@@ -376,13 +376,28 @@ struct ScoreSplit {
   int P;        // CTAs = min(U, SC_GRID)
 };
 
-inline ScoreSplit score_split(long long BH, long long nQ, long long nK) {
+// The number of key chunks per group trades load balance (more, shorter units) against
+// the centroid reload at every unit (measured on B200 at about two tiles of time): choose
+// the count that minimises (units of the busiest CTA) x (tiles per unit + 2) for a tensor
+// of BH_choice heads.  A launch over a slice of heads passes the whole tensor's head count,
+// so its chunks -- and with them the rounding of S -- are those of the whole launch.
+inline ScoreSplit score_split(long long BH, long long nQ, long long nK, long long BH_choice) {
   ScoreSplit s;
   s.G = (int)((nQ + SC_QB - 1) / SC_QB);
   s.T = (int)((nK + 127) / 128);
-  const int k = s.T < SC_MAX_CHUNKS ? s.T : SC_MAX_CHUNKS;
-  s.CT = (s.T + k - 1) / k;
-  s.KC = (s.T + s.CT - 1) / s.CT;
+  const long long R = BH_choice * s.G;
+  long long best = -1;
+  for (int k = 1; k <= SC_MAX_CHUNKS && k <= s.T; ++k) {
+    const int ct = (s.T + k - 1) / k;
+    const int kc = (s.T + ct - 1) / ct;
+    const long long per_cta = (R * kc + SC_GRID - 1) / SC_GRID;
+    const long long cost = per_cta * (ct + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      s.CT = ct;
+      s.KC = kc;
+    }
+  }
   s.U = BH * s.G * s.KC;
   s.P = (int)(s.U < SC_GRID ? s.U : SC_GRID);
   return s;
