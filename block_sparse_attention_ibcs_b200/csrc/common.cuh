@@ -136,18 +136,6 @@ AB_DEV void mbar_arrive_cpasync(uint64_t* bar) {
                : "memory");
 }
 
-AB_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Non-blocking probe of the phase with the given parity (no suspend hint).
 AB_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -217,7 +205,6 @@ AB_DEV void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
-AB_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 AB_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to async-proxy readers

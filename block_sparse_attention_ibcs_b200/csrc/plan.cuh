@@ -15,15 +15,17 @@
 //   its interval, with U = word 0 of Philox4x32-10(key = seed, counter = (row, offset_lo,
 //   offset_hi, 0)).
 //
-// One CTA of PLAN_THREADS threads per row.  The row is staged in shared memory when it
-// fits, otherwise re-read from global memory (L2) on each pass.  Passes over the row:
-// staging with the positive count and sum; F at lambda0 = s / sum(S) (with the sum of the
-// unsaturated scores) and at one Newton step from it -- these bracket lambda* to one ulp
-// on typical rows, otherwise a doubling search and bisection follow; and the output pass.
-// After staging every pass walks the thread's contiguous chunk, so F(lambda*) already gives
-// each thread its saturated count and q sum; the number drawn in a chunk needs no pass:
-// non-saturated intervals are shorter than 2^32, so the chunk's blocks hold exactly the
-// lattice points of the chunk's (contiguous) interval.
+// One CTA of PLAN_THREADS threads per row.  The row is staged in shared memory (one bulk
+// copy) when it fits, otherwise re-read from global memory (L2) on each pass.  Passes over
+// the row: staging with the positive count and sum; F at the three fp32 neighbours of
+// lambda0 = s / sum(S) (with the sum of the scores unsaturated at lambda0) -- without
+// saturation lambda* is lambda0 or its upper neighbour, so this one pass brackets it --
+// then, for the rows it does not bracket, a Newton step, doubling steps and bisection;
+// and the output pass.  After staging every pass walks the thread's contiguous chunk, so
+// the evaluation at lambda* already gives each thread its saturated count and q sum; the
+// number drawn before a chunk needs no pass: non-saturated intervals are shorter than
+// 2^32, so the blocks before it hold exactly the lattice points of their (contiguous)
+// interval.
 #pragma once
 
 #include "common.cuh"
@@ -84,44 +86,6 @@ AB_DEV bool fixed_q32(float lam, float sv, uint32_t& q) {
   const uint32_t b = __float_as_uint(x);
   q = __funnelshift_rc((b << 8) | 0x80000000u, 0u, 126u - (b >> 23));
   return x >= 1.0f;
-}
-
-// F's per-thread part: saturated blocks add 2^32, the others q_j.
-AB_DEV void add_q(float lam, float sv, uint64_t& acc) {
-  uint32_t q;
-  const bool sat = fixed_q32(lam, sv, q);
-  acc += sat ? TWO32 : (uint64_t)q;
-}
-
-// Block-wide sum of a uint64 (all threads get the result).  red: PLAN_WARPS slots.
-AB_DEV uint64_t block_sum_u64(uint64_t v, uint64_t* red) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  uint64_t tot = 0;
-#pragma unroll
-  for (int i = 0; i < PLAN_WARPS; ++i) tot += red[i];
-  return tot;
-}
-
-// Block-wide sums of a (uint64 count, fp64 value) pair, one pair of barriers.
-AB_DEV void block_sum_cd(uint64_t& c, double& v, uint64_t* redc, double* redv) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    c += __shfl_xor_sync(0xffffffffu, c, o);
-    v += __shfl_xor_sync(0xffffffffu, v, o);
-  }
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
-  if (l == 0) { redc[w] = c; redv[w] = v; }
-  __syncthreads();
-  c = 0;
-  v = 0.0;
-#pragma unroll
-  for (int i = 0; i < PLAN_WARPS; ++i) { c += redc[i]; v += redv[i]; }
 }
 
 // Exclusive block scans of two uint64 values in thread order, one pair of barriers;
