@@ -538,38 +538,63 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     uint64_t o = out_before;
     int32_t* oidx = a.idx + (size_t)row * a.s;
     uint32_t* oraw = reinterpret_cast<uint32_t*>(a.logpi + (size_t)row * a.s);
-    for (int i = c0; i < c1; ++i) {
-      const float4 v = load4(i);
-      const float x4[4] = {v.x, v.y, v.z, v.w};
+    if (reachable && !capped) {
+      // the common case, branch-light: a saturated block has q = 0 here and is drawn; a
+      // block past the row's end (score 0, q = 0) never is
+      uint32_t o32 = (uint32_t)out_before;
+      const uint32_t s32 = (uint32_t)a.s;
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = 4 * i + k;
-        if (j >= nK) break;
-        bool sel;
-        uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
-        if (reachable) {
+        for (int k = 0; k < 4; ++k) {
           uint32_t q;
-          if (fixed_q32(lam, x4[k], q)) {
-            sel = true;
-          } else if (!capped) {
-            sel = dist < q;
-            qq = q;
-            dist -= q;
-          } else {
-            const uint64_t st = min(pos, target), en = min(pos + q, target);
-            sel = below(en) != below(st);
-            qq = (uint32_t)(en - st);
-            pos += q;
+          const bool sat = fixed_q32(lam, x4[k], q);
+          const bool sel = sat || dist < q;
+          dist -= q;
+          if (sel) {
+            if (o32 < s32) {
+              oidx[o32] = 4 * i + k;
+              oraw[o32] = sat ? 0xFFFFFFFFu : q;  // pi = 1, or q (at most 2^32 - 256)
+            }
+            ++o32;
           }
-        } else {
-          sel = (x4[k] > 0.f) || (zero_i++ < need);
         }
-        if (sel) {
-          if (o < s) {
-            oidx[o] = j;
-            oraw[o] = qq;
+      }
+    } else {
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int j = 4 * i + k;
+          if (j >= nK) break;
+          bool sel;
+          uint32_t qq = 0xFFFFFFFFu;  // pi = 1 (a capped or ordinary q is at most 2^32 - 256)
+          if (reachable) {
+            uint32_t q;
+            if (fixed_q32(lam, x4[k], q)) {
+              sel = true;
+            } else if (!capped) {
+              sel = dist < q;
+              qq = q;
+              dist -= q;
+            } else {
+              const uint64_t st = min(pos, target), en = min(pos + q, target);
+              sel = below(en) != below(st);
+              qq = (uint32_t)(en - st);
+              pos += q;
+            }
+          } else {
+            sel = (x4[k] > 0.f) || (zero_i++ < need);
           }
-          ++o;
+          if (sel) {
+            if (o < s) {
+              oidx[o] = j;
+              oraw[o] = qq;
+            }
+            ++o;
+          }
         }
       }
     }
