@@ -24,10 +24,12 @@
 //              O += P_t V_t            (M=128, N=d, K=128; A = P from tensor memory, B = V
 //                                       read MN-major from the same tile layout)
 //   warps 0-3  softmax: thread r owns query row r = TMEM lane r.  Loads its Q row into
-//              tensor memory once, then per tile reads S (already shifted), keeps a lazy
-//              online max (raised only when a tile exceeds it by more than 2^8, decided
-//              per warp), writes P as bf16 into tensor memory, rescales its O row when
-//              the max moved, and finally writes O / l.
+//              tensor memory once, then per tile reads S (already shifted), takes the
+//              exponentials against a running reference max, writes P as bf16 into tensor
+//              memory and finally writes O / l.  The tile's maximum is computed only on a
+//              warp's first tile or when the tile's row sum passes 2^64; the reference is
+//              then raised (when the tile exceeds it by more than 2^8, decided per warp),
+//              P written again and O rescaled.
 // The shift -log(pi_j) of a sampled block (in logit units: -log(pi_j) * sqrt(d)) enters
 // through the tensor cores as one more K=16 step: A = [1 1 0 ... 0] for every query row,
 // B row n = [hi_n lo_n 0 ... 0] with hi = bf16(shift), lo = bf16(shift - hi), so S gains
@@ -50,6 +52,7 @@ constexpr int ATTN_ROW_GROUPS = ATTN_PRODUCERS / 16;  // 14: thread p copies row
 constexpr int ATTN_STAGES = 3;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
+constexpr float LSUM_LIMIT = 18446744073709551616.0f;  // 2^64: a tile's row sum above it takes the max path
 constexpr uint32_t SHIFT_PAD_BITS = 0xF180u;  // bf16 -2^100
 constexpr float PAD_LOGIT_LOG2 = -1e20f;      // a tile maximum below this is all padding
 
@@ -421,29 +424,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       mbar_arrive(&bars[B_SFREE]);
       if (r == 0) ev(EV_SM_LOADED, t);
       const float* z = reinterpret_cast<const float*>(zr);
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = z[k];
-#pragma unroll
-      for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], z[k]);
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
-      if (mt < PAD_LOGIT_LOG2) mt = -INFINITY;  // every column of the tile is padding
-      // Lazy rescale, decided per warp: tcgen05.ld/st are warp-collective, so when any
-      // row of the warp has to raise its reference max, every row of the warp moves to
-      // max(m_run, mt) (alpha = 1 where nothing changes) and the warp rescales O.
-      const bool need = mt > m_run + LAZY_RESCALE_LOG2;  // always true on a row's first finite tile
-      const bool rescale = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (rescale) {
-        const float m_new = fmaxf(mt, m_run);
-        if (m_new != -INFINITY) {
-          alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
-          m_run = m_new;
-        }
-      }
-      const float nmref = (m_run == -INFINITY) ? 0.f : -m_run;
-      if (r == 0) ev(EV_SM_MAX, t);
       // P buffer st is free once PV(t-2) has completed
       if (t >= 2) {
         ok = mbar_wait(&bars[B_PVDONE0 + st], ((t >> 1) - 1) & 1, abort_flag, a.timeout_ns);
@@ -452,26 +432,62 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       }
       if (r == 0) ev(EV_SM_PBUF, t);
       const uint32_t padr = (st ? TM_P1 : TM_P0) + lane_off;
-      float ls[8];
+      // P = exp2(z c + nm) as packed bf16 pairs into tensor memory; returns the row sum
+      auto emit = [&](float nm) {
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
+        for (int g = 0; g < 4; ++g) {  // 32 keys -> 16 TMEM columns of packed bf16 pairs
+          uint32_t pk[16];
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {  // 64 keys -> 32 TMEM columns of packed bf16 pairs
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c0 = 64 * g + 2 * e;
-          const float x0 = fmaf(z[c0], c, nmref);
-          const float x1 = fmaf(z[c0 + 1], c, nmref);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          ls[(2 * e) & 7] += p0;
-          ls[(2 * e + 1) & 7] += p1;
-          pk[e] = pack_bf16x2_rn(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * g + 2 * e;
+            const float p0 = fast_exp2(fmaf(z[c0], c, nm));
+            const float p1 = fast_exp2(fmaf(z[c0 + 1], c, nm));
+            ls[(2 * e) & 3] += p0;
+            ls[(2 * e + 1) & 3] += p1;
+            pk[e] = pack_bf16x2_rn(p0, p1);
+          }
+          tmem_st_32x32b_x16(padr + 16 * g, pk);
         }
-        tmem_st_32x32b_x32(padr + 32 * g, pk);
+        return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      };
+      // The exponentials are taken against the running reference m_run first; the tile's
+      // maximum is needed only on a warp's first tile, or when a value came out more than
+      // 2^57 above the reference (the row sum passes 2^64, or overflowed).  Values up to
+      // 2^64 keep every sum far inside fp32 range, and softmax weights do not depend on the
+      // reference, so the output is the same softmax.  Decided per warp: tcgen05.ld/st are
+      // warp-collective, so when any row of the warp has to raise its reference, every row
+      // of the warp moves to max(m_run, tile max) (alpha = 1 where nothing changes), its P
+      // row is written again and the warp rescales O.
+      float alpha = 1.f;
+      bool rescale = false;
+      float lsum = 0.f;
+      bool redo = __any_sync(0xffffffffu, m_run == -INFINITY);
+      if (!redo) {
+        lsum = emit(-m_run);
+        redo = __any_sync(0xffffffffu, !(lsum <= LSUM_LIMIT));
       }
-      const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      if (redo) {
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = z[k];
+#pragma unroll
+        for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], z[k]);
+        float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+        if (mt < PAD_LOGIT_LOG2) mt = -INFINITY;  // every column of the tile is padding
+        const bool need = mt > m_run + LAZY_RESCALE_LOG2;  // always true on a row's first finite tile
+        rescale = __any_sync(0xffffffffu, need);
+        if (rescale) {
+          const float m_new = fmaxf(mt, m_run);
+          if (m_new != -INFINITY) {
+            alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
+            m_run = m_new;
+          }
+        }
+        lsum = emit((m_run == -INFINITY) ? 0.f : -m_run);
+      }
+      if (r == 0) ev(EV_SM_MAX, t);
       l_run = l_run * alpha + lsum;
       if (rescale && t > 0) {  // warp-uniform; O holds no data before PV(0)
         // O is stable once PV(t-1) has completed
