@@ -166,7 +166,7 @@ def gathered_bytes(w):
 # DRAM bytes per attention launch from the newest ncu capture of the current kernel
 # (dram__bytes_read.sum + dram__bytes_write.sum, scaled from the captured shape to the
 # bench shape by the number of heads); None while the kernel differs from the captured one.
-ATTN_TRAFFIC_BYTES = 3.463e9  # ncu dram bytes of one Wan2.1-1.3B launch (1.0390 GB) x 40/12 heads
+ATTN_TRAFFIC_BYTES = 3.457e9  # ncu dram bytes of one Wan2.1-1.3B launch (1.0371 GB) x 40/12 heads
 
 
 def select_plan_bytes(w):

@@ -5,6 +5,8 @@
 //   cpasync : 16-byte cp.async per thread (the attention kernel's copy), 8 warps, one
 //             32 KB tile in flight per CTA
 //   bulk<NT>: 1 KB cp.async.bulk copies completing on an mbarrier, NT tiles in flight
+//   pipe<NST>: the attention kernel's pattern: 4 to 16 warps, K and V of a 128-token tile
+//             per 64 KB stage, NST stages in flight, footprints of 16, 40 and 64 MB
 //
 // Prints cycles per 32 KB tile, bytes/cycle per SM and in aggregate, for grids of 148
 // (one CTA per SM), 74 and 37 CTAs.  Block indices come from a fixed LCG; every address
@@ -81,6 +83,45 @@ __global__ void gather_bulk(const uint8_t* __restrict__ g, const int* __restrict
   if (tid == 0) out[blockIdx.x] = clock64() - t0;
 }
 
+// The attention kernel's own pattern: W copying warps; a stage is one 128-token tile of K
+// and of V (the same 32 block indices into a K half and a V half of a footprint of F bytes,
+// 64 KB per stage); NST stages in flight (cp.async groups), so the copy rate rather than one
+// tile's latency is measured.  As in the kernel, each warp loads a tile's 32 block indices
+// with one coalesced load a tile ahead and hands them to the copying lanes by shuffles; the
+// random words map into the footprint by a multiply-high.
+template <int NST>
+__global__ void gather_pipe(const uint8_t* __restrict__ g, const uint32_t* __restrict__ blocks, int nb,
+                            int iters, size_t half_bytes, long long* out) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sbase = sa(sm);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nthr = blockDim.x;
+  const uint32_t nblk = (uint32_t)(half_bytes / 1024);
+  const int per_thread = (4096 + nthr - 1) / nthr;  // warp-uniform trip count
+  uint32_t cur = blocks[(blockIdx.x * iters * 32 + lane) & (nb - 1)];
+  const long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    const uint32_t nxt = blocks[((blockIdx.x * iters + it + 1) * 32 + lane) & (nb - 1)];
+    const uint32_t stage = sbase + (uint32_t)(it % NST) * 65536u;
+    for (int k = 0; k < per_thread; ++k) {
+      const int c = tid + k * nthr;
+      const int kv = (c >> 11) & 1, r = (c >> 4) & 127, u = c & 15;
+      const uint32_t blk = __umulhi(__shfl_sync(0xffffffffu, cur, r >> 2), nblk);
+      if (c < 4096) {
+        const uint8_t* src = g + (size_t)kv * half_bytes + ((size_t)blk * 4 + (r & 3)) * 256 + u * 16;
+        const uint32_t dst = stage + kv * 32768u + (u >> 3) * 16384 + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      }
+    }
+    cur = nxt;
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group %0;" ::"n"(NST - 1) : "memory");
+    __syncthreads();
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  if (tid == 0) out[blockIdx.x] = clock64() - t0;
+}
+
 }  // namespace
 
 int main() {
@@ -124,6 +165,38 @@ int main() {
     report("bulk x1", grid);
     for (int rep = 0; rep < 2; ++rep) gather_bulk<4><<<grid, 32, 128 * 1024>>>(g, blocks, (int)hb.size(), iters, out, err);
     report("bulk x4", grid);
+  }
+  // the attention pattern: K+V stages of 64 KB, footprints from 16 MB to the whole 64 MB,
+  // 4 to 16 copying warps
+  std::vector<uint32_t> hr(1u << 20);
+  for (auto& v : hr) v = (x = x * 1664525u + 1013904223u);
+  uint32_t* rnd;
+  cudaMalloc(&rnd, hr.size() * 4);
+  cudaMemcpy(rnd, hr.data(), hr.size() * 4, cudaMemcpyHostToDevice);
+  cudaFuncSetAttribute(gather_pipe<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(gather_pipe<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+  for (size_t mb : {16, 40, 64}) {
+    const size_t half = (mb << 20) / 2;
+    for (int warps : {4, 7, 12, 16}) {
+      auto report_pipe = [&](const char* name) {
+        cudaDeviceSynchronize();
+        std::vector<long long> h(148);
+        cudaMemcpy(h.data(), out, 148 * 8, cudaMemcpyDeviceToHost);
+        double avg = 0;
+        for (auto v : h) avg += (double)v;
+        avg /= 148;
+        printf("footprint %2zu MB %2d warps %-8s %7.0f cycles/64KB stage  %5.1f B/cycle/SM  aggregate %6.0f B/cycle\n",
+               mb, warps, name, avg / iters, 65536.0 * iters / avg, 148 * 65536.0 * iters / avg);
+      };
+      if (mb == 40) {
+        for (int rep = 0; rep < 2; ++rep)
+          gather_pipe<1><<<148, warps * 32, 64 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out);
+        report_pipe("pipe x1");
+      }
+      for (int rep = 0; rep < 2; ++rep)
+        gather_pipe<3><<<148, warps * 32, 192 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out);
+      report_pipe("pipe x3");
+    }
   }
   int herr = 0;
   cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);

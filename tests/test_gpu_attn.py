@@ -110,6 +110,34 @@ def test_all_blocks_packed_equals_dense_path_bitwise(bk):
     assert torch.equal(O1, O2)
 
 
+@pytest.mark.parametrize("spike_nats", [38.0, 60.0])
+def test_late_logit_spikes(spike_nats):
+    """Logits far above the first tile's maximum in later tiles, for warp 0 of a query block.
+
+    The softmax takes its exponentials against the running reference and falls back to
+    the tile maximum (with a rescale of O) only when a tile's row sum passes 2^64.  With
+    a spike of 38 nats (about 2^55 over the reference) every tile stays on the fast path
+    with P values near 2^52; with 60 nats the tile holding it (tile 5) takes the fallback
+    after an intermediate spike of 36 nats in tile 3 that does not.  Warps 1-3 of the
+    block have no spike, so the fallback is exercised per warp."""
+    H, N, d, bk = 1, 1024, 64, 4
+    nK = N // bk
+    Q, K, V = _qkv(H, N, d, seed=11)
+    g = torch.Generator().manual_seed(7)
+    u = (torch.randint(0, 2, (d,), generator=g) * 2 - 1).float()  # |u|^2 = d
+    beta = spike_nats * math.sqrt(d) / d  # (beta u) . u / sqrt(d) = spike_nats
+    Q[0, 0, :32] = u.bfloat16()
+    K[0, 0, 5 * 128 + 7] = (beta * u).bfloat16()
+    K[0, 0, 3 * 128 + 9] = (0.6 * beta * u).bfloat16()
+    p = ab.params(1, H, N, d, kv_block=bk)
+    idx = torch.arange(nK, dtype=torch.int32).repeat(H * 8, 1)
+    lp = torch.zeros(H * 8, nK)
+    O_ = _run(p, Q, K, V, idx, lp, nK)
+    _check(O_, Q, K, V, idx, lp, H, N, bk, qblocks=[0, 1])
+    # the spike dominates warp 0's rows (the rest of the row's mass is below e^-20)
+    assert np.abs(np64(O_[0, 0, :32]) - np64(V[0, 0, 5 * 128 + 7])).max() < 1e-2
+
+
 def test_bad_index_status():
     H, N, d, bk, s = 1, 256, 64, 4, 8
     Q, K, V = _qkv(H, N, d, seed=9)
