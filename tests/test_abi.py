@@ -51,6 +51,9 @@ def test_workspace_bytes():
     (dict(d=96), -2), (dict(d=0), -1), (dict(q_block=64), -2), (dict(kv_block=3), -1),
     (dict(kv_block=256), -1), (dict(clusters=0), -1), (dict(clusters=9), -2),
     (dict(kmeans_iters=-1), -1), (dict(kmeans_iters=5), -2), (dict(N=0), -1),
+    (dict(B=0), -1), (dict(H=0), -1), (dict(B=-3), -1),
+    # size limits: (b, h, query block) CTAs must fit a 1-D grid, nK * 2^32 a uint64
+    (dict(B=1, H=4_000_000, N=75600), -2), (dict(N=(1 << 31) - 1, kv_block=1), -2),
 ])
 def test_bad_params_rejected(bad, code):
     kw = dict(B=1, H=2, N=1024, d=64, kv_block=4, clusters=8, kmeans_iters=1, q_block=128)
@@ -59,6 +62,17 @@ def test_bad_params_rejected(bad, code):
                     kw["clusters"], kw["kmeans_iters"])
     n = ctypes.c_size_t(0)
     assert ab.lib().ab_workspace_bytes(ctypes.byref(p), ctypes.byref(n)) == code
+
+
+def test_largest_accepted_grid():
+    # BH * nQ = 2^31 - 1 exactly is accepted (one CTA per (b, h, query block))
+    nQ = 591
+    H = ((1 << 31) - 1) // nQ
+    p = ab.params(1, H, 75600, 128)
+    n = ctypes.c_size_t(0)
+    assert ab.lib().ab_workspace_bytes(ctypes.byref(p), ctypes.byref(n)) == 0
+    p = ab.params(1, H + 1, 75600, 128)
+    assert ab.lib().ab_workspace_bytes(ctypes.byref(p), ctypes.byref(n)) == -2
 
 
 def test_null_and_misaligned_pointers_rejected_before_any_cuda_call():
