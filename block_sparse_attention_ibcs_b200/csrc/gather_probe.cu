@@ -89,9 +89,9 @@ __global__ void gather_bulk(const uint8_t* __restrict__ g, const int* __restrict
 // tile's latency is measured.  As in the kernel, each warp loads a tile's 32 block indices
 // with one coalesced load a tile ahead and hands them to the copying lanes by shuffles; the
 // random words map into the footprint by a multiply-high.
-template <int NST>
+template <int NST, int EXTRA = 0>
 __global__ void gather_pipe(const uint8_t* __restrict__ g, const uint32_t* __restrict__ blocks, int nb,
-                            int iters, size_t half_bytes, long long* out) {
+                            int iters, size_t half_bytes, long long* out, uint32_t zero = 0) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sbase = sa(sm);
   const int tid = threadIdx.x, lane = tid & 31;
@@ -106,7 +106,10 @@ __global__ void gather_pipe(const uint8_t* __restrict__ g, const uint32_t* __res
     for (int k = 0; k < per_thread; ++k) {
       const int c = tid + k * nthr;
       const int kv = (c >> 11) & 1, r = (c >> 4) & 127, u = c & 15;
-      const uint32_t blk = __umulhi(__shfl_sync(0xffffffffu, cur, r >> 2), nblk);
+      uint32_t blk = __umulhi(__shfl_sync(0xffffffffu, cur, r >> 2), nblk);
+#pragma unroll
+      for (int x = 0; x < EXTRA; ++x)  // EXTRA integer instructions per copy (zero is 0)
+        asm volatile("xor.b32 %0, %0, %1;" : "+r"(blk) : "r"(zero));
       if (c < 4096) {
         const uint8_t* src = g + (size_t)kv * half_bytes + ((size_t)blk * 4 + (r & 3)) * 256 + u * 16;
         const uint32_t dst = stage + kv * 32768u + (u >> 3) * 16384 + r * 128 + (((u & 7) ^ (r & 7)) << 4);
@@ -197,6 +200,31 @@ int main() {
         gather_pipe<3><<<148, warps * 32, 192 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out);
       report_pipe("pipe x3");
     }
+  }
+  // sensitivity of the copy rate to the instructions spent per copy (7 warps, 40 MB, 3 stages)
+  cudaFuncSetAttribute(gather_pipe<3, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+  cudaFuncSetAttribute(gather_pipe<3, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+  {
+    const size_t half = (40ull << 20) / 2;
+    auto rep_x = [&](int extra) {
+      cudaDeviceSynchronize();
+      std::vector<long long> h(148);
+      cudaMemcpy(h.data(), out, 148 * 8, cudaMemcpyDeviceToHost);
+      double avg = 0;
+      for (auto v : h) avg += (double)v;
+      avg /= 148;
+      printf("footprint 40 MB  7 warps pipe x3 +%d int ops/copy %7.0f cycles/64KB stage  %5.1f B/cycle/SM\n", extra,
+             avg / iters, 65536.0 * iters / avg);
+    };
+    for (int rep = 0; rep < 2; ++rep)
+      gather_pipe<3, 0><<<148, 224, 192 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out, 0u);
+    rep_x(0);
+    for (int rep = 0; rep < 2; ++rep)
+      gather_pipe<3, 4><<<148, 224, 192 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out, 0u);
+    rep_x(4);
+    for (int rep = 0; rep < 2; ++rep)
+      gather_pipe<3, 8><<<148, 224, 192 * 1024>>>(g, rnd, (int)hr.size(), iters, half, out, 0u);
+    rep_x(8);
   }
   int herr = 0;
   cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);
