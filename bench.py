@@ -426,18 +426,34 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def oracle_threads():
+    """Threads the oracle's numpy work runs on: the BLAS thread pool (threadpoolctl), else
+    torch's intra-op thread count."""
+    try:
+        import threadpoolctl
+
+        n = [i.get("num_threads", 0) for i in threadpoolctl.threadpool_info()
+             if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    import torch
+
+    return torch.get_num_threads()
+
+
 def cpu_baseline(w, seconds=15.0):
     """The oracle as it stands on the host cores: select + plan + attention for a bounded
     sample of query blocks of head 0, expressed in the metric's unit (kept-block FLOP/s)."""
     import numpy as np
-    import torch
 
     from block_sparse_attention_ibcs_b200.inputs import make_qkv
     from oracle import abattn_oracle as O
 
     Q, K, V = make_qkv(w, device="cpu", heads=[0])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
-    cores = torch.get_num_threads()
+    cores = oracle_threads()
     t0 = time.perf_counter()
     Kp = O.pool_keys(k, w.kv_block)
     done = 0
