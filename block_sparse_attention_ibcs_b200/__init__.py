@@ -106,6 +106,34 @@ def _ptr(t, name, dtype=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _sizes(p):
+    """(B*H, nQ, nK) of a parameter set, or None when the parameters are invalid (the
+    library then reports that itself)."""
+    if p is None or min(p.B, p.H, p.N, p.d, p.kv_block) < 1:
+        return None
+    return p.B * p.H, -(-p.N // 128), -(-p.N // p.kv_block)
+
+
+def _need(p, **bufs):
+    """Every given tensor holds at least the elements the call reads or writes through its
+    pointer; ``bufs`` maps a name to (tensor, count as a function of (BH, nQ, nK)).  A smaller
+    buffer would send the kernels past its end, so it is refused here."""
+    dims = _sizes(p)
+    if dims is None:
+        return
+    for name, (t, count) in bufs.items():
+        if t is None:
+            continue
+        n = int(count(*dims))
+        if t.numel() < n:
+            raise ValueError(f"{name} holds {t.numel()} elements; the call needs {n}")
+
+
+def _qkv(p, *names_tensors):
+    """Size rules for [B,H,N,d] tensors."""
+    return {n: (t, lambda bh, nq, nk: bh * p.N * p.d) for n, t in names_tensors}
+
+
 def _check(code: int, where: str):
     if code != AB_OK:
         raise ABError(code, where)
@@ -128,6 +156,8 @@ def ab_workspace_bytes(p: ABParams) -> int:
 def ab_select(p, Q, K, S, ws, stream=None):
     import torch
 
+    _need(p, **_qkv(p, ("Q", Q), ("K", K)), S=(S, lambda bh, nq, nk: bh * nq * nk))
+
     _check(lib().ab_select(ctypes.byref(p), _ptr(Q, "Q", torch.bfloat16), _ptr(K, "K", torch.bfloat16),
                            _ptr(S, "S", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
                            _stream(stream)), "ab_select")
@@ -135,6 +165,12 @@ def ab_select(p, Q, K, S, ws, stream=None):
 
 def ab_select_debug(p, Q, K, S, ws, labels=None, cent=None, w=None, Kp=None, stream=None):
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K)), S=(S, lambda bh, nq, nk: bh * nq * nk),
+          labels=(labels, lambda bh, nq, nk: bh * nq * 128),
+          cent=(cent, lambda bh, nq, nk: bh * nq * p.clusters * p.d),
+          w=(w, lambda bh, nq, nk: bh * nq * p.clusters),
+          Kp=(Kp, lambda bh, nq, nk: bh * nk * p.d))
 
     _check(lib().ab_select_debug(
         ctypes.byref(p), _ptr(Q, "Q", torch.bfloat16), _ptr(K, "K", torch.bfloat16),
@@ -147,6 +183,9 @@ def ab_select_debug(p, Q, K, S, ws, labels=None, cent=None, w=None, Kp=None, str
 def ab_plan(p, S, s, seed, offset, idx, logpi, stream=None):
     import torch
 
+    _need(p, S=(S, lambda bh, nq, nk: bh * nq * nk), idx=(idx, lambda bh, nq, nk: bh * nq * s),
+          logpi=(logpi, lambda bh, nq, nk: bh * nq * s))
+
     _check(lib().ab_plan(ctypes.byref(p), _ptr(S, "S", torch.float32), int(s), int(seed), int(offset),
                          _ptr(idx, "idx", torch.int32), _ptr(logpi, "logpi", torch.float32),
                          _stream(stream)), "ab_plan")
@@ -156,6 +195,9 @@ def ab_select_plan(p, Q, K, S, ws, s, seed, offset, idx, logpi, groups=0, stream
                    stream2=None):
     """ab_select then ab_plan, overlapped across head groups on ``stream`` and ``stream2``."""
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K)), S=(S, lambda bh, nq, nk: bh * nq * nk),
+          idx=(idx, lambda bh, nq, nk: bh * nq * s), logpi=(logpi, lambda bh, nq, nk: bh * nq * s))
 
     _check(lib().ab_select_plan(ctypes.byref(p), _ptr(Q, "Q", torch.bfloat16),
                                 _ptr(K, "K", torch.bfloat16), _ptr(S, "S", torch.float32),
@@ -170,6 +212,9 @@ def ab_plan_variant(p, S, s, seed, offset, mode, idx, logpi, stream=None):
     "uniform"."""
     import torch
 
+    _need(p, S=(S, lambda bh, nq, nk: bh * nq * nk), idx=(idx, lambda bh, nq, nk: bh * nq * s),
+          logpi=(logpi, lambda bh, nq, nk: bh * nq * s))
+
     m = PLAN_MODES[mode] if isinstance(mode, str) else int(mode)
     _check(lib().ab_plan_variant(ctypes.byref(p), _ptr(S, "S", torch.float32), int(s), int(seed),
                                  int(offset), m, _ptr(idx, "idx", torch.int32),
@@ -180,6 +225,9 @@ def ab_plan_variant(p, S, s, seed, offset, mode, idx, logpi, stream=None):
 def ab_sample(p, pi, s, seed, offset, idx, logpi, stream=None):
     import torch
 
+    _need(p, pi=(pi, lambda bh, nq, nk: bh * nq * nk), idx=(idx, lambda bh, nq, nk: bh * nq * s),
+          logpi=(logpi, lambda bh, nq, nk: bh * nq * s))
+
     _check(lib().ab_sample(ctypes.byref(p), _ptr(pi, "pi", torch.float32), int(s), int(seed),
                            int(offset), _ptr(idx, "idx", torch.int32),
                            _ptr(logpi, "logpi", torch.float32), _stream(stream)), "ab_sample")
@@ -187,6 +235,9 @@ def ab_sample(p, pi, s, seed, offset, idx, logpi, stream=None):
 
 def ab_attn(p, Q, K, V, idx, logpi, s, O, stream=None):
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K), ("V", V), ("O", O)),
+          idx=(idx, lambda bh, nq, nk: bh * nq * s), logpi=(logpi, lambda bh, nq, nk: bh * nq * s))
 
     bf = torch.bfloat16
     _check(lib().ab_attn(ctypes.byref(p), _ptr(Q, "Q", bf), _ptr(K, "K", bf), _ptr(V, "V", bf),
@@ -196,6 +247,8 @@ def ab_attn(p, Q, K, V, idx, logpi, s, O, stream=None):
 
 def ab_attn_dense(p, Q, K, V, O, stream=None):
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K), ("V", V), ("O", O)))
 
     bf = torch.bfloat16
     _check(lib().ab_attn_dense(ctypes.byref(p), _ptr(Q, "Q", bf), _ptr(K, "K", bf), _ptr(V, "V", bf),
@@ -207,6 +260,10 @@ def ab_attn_debug(p, Q, K, V, idx, logpi, s, O, skip_first_arrival, timeout_ns, 
     """Test/profiling hook: ab_attn with a producer arrival skipped, another device wait
     limit, and optionally a per-tile clock64 event trace (int64 tensor of 3*16*128)."""
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K), ("V", V), ("O", O)),
+          idx=(idx, lambda bh, nq, nk: bh * nq * s), logpi=(logpi, lambda bh, nq, nk: bh * nq * s),
+          trace=(trace, lambda bh, nq, nk: 3 * 16 * 128))
 
     bf = torch.bfloat16
     _check(lib().ab_attn_debug(ctypes.byref(p), _ptr(Q, "Q", bf), _ptr(K, "K", bf), _ptr(V, "V", bf),
@@ -227,6 +284,8 @@ def ab_select_noalloc(p, Q, K, S, stream=None):
     Calls that overlap on the GPU share that scratch and race; serialise them.
     """
     import torch
+
+    _need(p, **_qkv(p, ("Q", Q), ("K", K)), S=(S, lambda bh, nq, nk: bh * nq * nk))
 
     f = lib().ab_select_noalloc
     f.argtypes = [_P, _vp, _vp, _vp, _vp]
