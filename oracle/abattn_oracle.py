@@ -121,8 +121,10 @@ def kmeans_block(Qb: np.ndarray, C: int = 8, iters: int = 1):
     contiguous segment means (R1); each iteration assigns every query to the
     nearest centroid in squared Euclidean distance (ties to the lowest index)
     and replaces each centroid by the mean of its members (R2).  gap is the
-    relative distance gap between the best and second-best centroid of the
-    last assignment (inf when there is no assignment).
+    relative distance gap (d2 - d1) / d2 between the best (d1) and second-best
+    (d2) live centroid of the last assignment; clusters emptied by an earlier
+    iteration take no part; inf when there is no assignment or only one live
+    cluster; 0 on an exact tie.
     """
     n, d = Qb.shape
     cent = np.zeros((C, d))
@@ -142,6 +144,7 @@ def kmeans_block(Qb: np.ndarray, C: int = 8, iters: int = 1):
         srt = np.sort(dist, axis=1)
         with np.errstate(invalid="ignore", divide="ignore"):
             gap = (srt[:, 1] - srt[:, 0]) / np.maximum(srt[:, 1], 1e-300)
+        gap[np.isinf(srt[:, 1])] = np.inf  # one live cluster: no runner-up, no near-tie
         new = np.zeros((C, d))
         counts = np.bincount(labels, minlength=C)
         for c in range(C):

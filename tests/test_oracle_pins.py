@@ -137,6 +137,76 @@ def test_kmeans_identical_queries():
     assert w[0] == 1.0 and (labels == 0).all() and np.array_equal(cent[0], q)
 
 
+def test_kmeans_gap_hand_example():
+    # n = 6 one-dimensional queries, 3 clusters: segments {0,2}, {-1,-3}, {9,11} have means
+    # 1, -2, 10.  Query 0 lies at squared distances 1, 4, 100: the best and the second best
+    # give (4 - 1) / 4 = 0.75 (the third distance must not enter).
+    Qb = np.array([[0.0], [2.0], [-1.0], [-3.0], [9.0], [11.0]])
+    _, _, labels, gap = O.kmeans_block(Qb, C=3, iters=1)
+    assert labels.tolist() == [0, 0, 1, 1, 2, 2]
+    # distances: q1 = 2: 1, 16, 64; q2 = -1: 4, 1, 121; q3 = -3: 16, 1, 169; q4 = 9: 64, 121,
+    # 1; q5 = 11: 100, 169, 1
+    assert gap.tolist() == [0.75, 15 / 16, 0.75, 15 / 16, 63 / 64, 99 / 100]
+
+
+def test_kmeans_gap_exact_tie_is_zero():
+    # segments {-3, 3}, {3, 9} have means 0 and 6; both queries at 3 are 9 from each mean:
+    # an exact tie (gap 0), resolved to the lower cluster.
+    Qb = np.array([[-3.0], [3.0], [3.0], [9.0]])
+    cent, w, labels, gap = O.kmeans_block(Qb, C=2, iters=1)
+    assert labels.tolist() == [0, 0, 0, 1]
+    assert gap.tolist() == [72 / 81, 0.0, 0.0, 72 / 81]
+    assert w.tolist() == [0.75, 0.25] and cent[:, 0].tolist() == [1.0, 9.0]
+
+
+def test_kmeans_gap_ignores_emptied_clusters():
+    # segments {0}, {10}, {9, 11}: means 0, 10, 10.  The first assignment sends 10, 9 and 11
+    # to cluster 1 (ties to the lower index), so cluster 2 empties.  In the second
+    # assignment query 9 is 81 from cluster 0 and 1 from cluster 1; the emptied cluster
+    # (its old mean 10 would also be at distance 1) must not count: gap = 80/81, not 0.
+    Qb = np.array([[0.0], [10.0], [9.0], [11.0]])
+    cent, w, labels, gap = O.kmeans_block(Qb, C=3, iters=2)
+    assert labels.tolist() == [0, 1, 1, 1]
+    assert w.tolist() == [0.25, 0.75, 0.0]
+    assert cent[:, 0].tolist() == [0.0, 10.0, 0.0]
+    assert gap.tolist() == [1.0, 1.0, 80 / 81, 120 / 121]
+    # only one live cluster: no runner-up, so no near-tie
+    _, _, _, g1 = O.kmeans_block(np.array([[1.0], [1.0]]), C=2, iters=2)
+    assert np.isinf(g1).all()
+
+
+def test_scores_from_labels_hand_example():
+    # d = 1, two pooled keys 0 and 1.  Labels put query 1 (value 0) into cluster 1 with the
+    # two queries at 2: cluster 0 = {0} (mean 0, share 1/4), cluster 1 = {0, 2, 2} (mean 4/3,
+    # share 3/4).  4/3 = 1.0101010...b rounds to the bf16 value 1.0101011b = 1.3359375.
+    # With two keys each softmax is a logistic: cluster 0 gives (1/2, 1/2), cluster 1 gives
+    # (1 - p, p) with p = 1 / (1 + e^-1.3359375).
+    Qb = np.array([[0.0], [0.0], [2.0], [2.0]])
+    Kp = np.array([[0.0], [1.0]])
+    S = O.scores_from_labels(Qb, np.array([0, 1, 1, 1]), Kp, C=2)
+    p = 1.0 / (1.0 + math.exp(-1.3359375))
+    want = [0.25 * 0.5 + 0.75 * (1 - p), 0.25 * 0.5 + 0.75 * p]
+    assert S.dtype == np.float32
+    np.testing.assert_allclose(S, want, rtol=2e-7, atol=0)
+    # the unrounded mean 4/3 would be off by far more than the fp32 output rounding
+    p_raw = 1.0 / (1.0 + math.exp(-4.0 / 3.0))
+    assert abs(0.75 * (p - p_raw)) > 1e-4 * want[1]
+
+
+def test_scores_from_labels_reproduces_kmeans_scores():
+    # with the labels of the last assignment, the rebuilt centroids and shares are exactly
+    # kmeans_block's, so the score rows agree bit for bit (iterations 0, 1, 2; ragged n)
+    rng = np.random.default_rng(6)
+    Kp = O.bf16_round(rng.standard_normal((200, 32)))
+    for n in (128, 80, 13):
+        Qb = O.bf16_round(rng.standard_normal((n, 32)) + rng.integers(0, 4, (n, 1)))
+        for iters in (0, 1, 2):
+            cent, w, labels, _ = O.kmeans_block(Qb, 8, iters)
+            want = O.block_scores(cent, w, Kp).astype(np.float32)
+            got = O.scores_from_labels(Qb, labels, Kp, C=8)
+            assert np.array_equal(got, want), (n, iters)
+
+
 # ---------------------------------------------------------------- scores
 
 
