@@ -25,8 +25,7 @@ def nvcc_cmd(verbose_ptxas: bool = False):
 
 def sources():
     d = os.path.join(HERE, "csrc")
-    return ([os.path.join(d, f) for f in os.listdir(d) if f not in ("gather_probe.cu", "mufu_probe.cu")] +
-            [os.path.join(ROOT, "include", "abattn.h")])
+    return [os.path.join(d, f) for f in os.listdir(d)] + [os.path.join(ROOT, "include", "abattn.h")]
 
 
 def up_to_date() -> bool:
@@ -47,41 +46,6 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     return OUT
 
 
-PROBE_SRC = os.path.join(HERE, "csrc", "gather_probe.cu")
-PROBE_OUT = os.path.join(HERE, "gather_probe")
-
-
-def build_probe() -> str:
-    """The L2 gather-bandwidth probe (a stand-alone executable, not part of the library)."""
-    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", PROBE_SRC,
-           "-o", PROBE_OUT]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building gather_probe")
-    return PROBE_OUT
-
-
-MUFU_SRC = os.path.join(HERE, "csrc", "mufu_probe.cu")
-MUFU_OUT = os.path.join(HERE, "mufu_probe")
-
-
-def build_mufu_probe() -> str:
-    """The exponential-throughput probe (a stand-alone executable, not part of the library)."""
-    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
-           "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"), MUFU_SRC, "-o", MUFU_OUT]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building mufu_probe")
-    return MUFU_OUT
-
-
 if __name__ == "__main__":
-    if "--mufu-probe" in sys.argv:
-        print(build_mufu_probe())
-    elif "--probe" in sys.argv:
-        print(build_probe())
-    else:
-        build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
-        print(OUT)
+    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
+    print(OUT)
