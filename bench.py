@@ -8,14 +8,19 @@ One step = one pass of the whole hot path on the Wan2.1-14B-shaped layer
 Inputs are synthetic (random-Fourier Q/K + noise, Gaussian V), generated on the
 device before timing; every tensor is larger than L2, so no flush is needed.
 
-Multi-GPU (torchrun): weak scaling, every rank runs its own full layer (independent
-heads/batches need no exchange); the step time is the max over ranks.
+Multi-GPU (torchrun), sharded by heads with no data-path collective (every (b, h) is
+independent): by default a layer of H * N heads over N ranks, H heads each (weak scaling);
+with --shard strong the configured layer's H heads split over the ranks (strong scaling).
+Each rank calls the library on its own heads with head0 / heads_total set, so its S, plan
+and O equal the matching rows of a one-GPU run over the whole layer.  The step time is the
+max over ranks.
 
 --impl reference times the CPU oracle (the only reference implementation: the pages
 publish no code) on a bounded sample of the same workload, on rank 0.
 """
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -24,6 +29,8 @@ import subprocess
 import sys
 import threading
 import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -139,13 +146,6 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
-def rank_workload(w, rank):
-    """Weak scaling: rank r processes its own independent layer (same shape, own seed)."""
-    import dataclasses
-
-    return dataclasses.replace(w, seed=w.seed + 1000 * rank, philox_seed=w.philox_seed + 1000 * rank)
-
-
 def shard_heads(H, world, rank):
     """Head-parallel split of one layer: contiguous head range of this rank."""
     base, extra = divmod(H, world)
@@ -153,27 +153,58 @@ def shard_heads(H, world, rank):
     return lo, lo + base + (1 if rank < extra else 0)
 
 
-def kept_flops(w):
-    """Kept-block attention FLOPs of one ab_attn call: 4 * B * H * N * (s * bk) * d."""
-    return 4.0 * w.B * w.H * w.N * (w.s * w.kv_block) * w.d
+def rank_heads(w, world, rank, shard):
+    """(head0, head1, heads_total) of this rank.  "weak": a layer of w.H * world heads, w.H
+    per rank; "strong": the layer's w.H heads split over the ranks."""
+    if shard == "strong":
+        h0, h1 = shard_heads(w.H, world, rank)
+        return h0, h1, w.H
+    h0, h1 = shard_heads(w.H * world, world, rank)
+    return h0, h1, w.H * world
 
 
-def gathered_bytes(w):
+def kept_flops(w, heads=None):
+    """Kept-block attention FLOPs of one ab_attn call over `heads` heads (default w.H):
+    4 * B * heads * N * (s * bk) * d."""
+    return 4.0 * w.B * (w.H if heads is None else heads) * w.N * (w.s * w.kv_block) * w.d
+
+
+def gathered_bytes(w, heads=None):
     """K and V bytes one ab_attn call gathers: every query block reads s*bk tokens of each."""
-    return 2.0 * w.B * w.H * w.nQ * (w.s * w.kv_block) * w.d * 2
+    return 2.0 * w.B * (w.H if heads is None else heads) * w.nQ * (w.s * w.kv_block) * w.d * 2
 
 
-# DRAM bytes per attention launch from the newest ncu capture of the current kernel
-# (dram__bytes_read.sum + dram__bytes_write.sum, scaled from the captured shape to the
-# bench shape by the number of heads); None while the kernel differs from the captured one.
-ATTN_TRAFFIC_BYTES = 3.457e9  # ncu dram bytes of one Wan2.1-1.3B launch (1.0371 GB) x 40/12 heads
+def attn_source_sha256():
+    """Hash of the attention kernel's sources (the kernel and the helpers it inlines)."""
+    h = hashlib.sha256()
+    for f in ("attn.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_ibcs_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
-def select_plan_bytes(w):
+# DRAM bytes of one attention launch at the Wan2.1-14B shape from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum of the Wan2.1-1.3B-shaped launch, scaled by
+# the number of heads: every head's K, V, Q and O cross DRAM once), valid only for the
+# kernel source it was taken on; `roofline.traffic` is null for any other source.
+ATTN_TRAFFIC = {"bytes_wan14b": None, "captured_heads": 12, "source_sha256": None}
+
+
+def attn_traffic(w, heads):
+    t = ATTN_TRAFFIC
+    if t["bytes_wan14b"] is None or t["source_sha256"] != attn_source_sha256():
+        return None
+    if (w.N, w.d, w.s, w.kv_block) != (75600, 128, 2048, 4):
+        return None
+    return round(t["bytes_wan14b"] * heads / 40.0)
+
+
+def select_plan_bytes(w, heads=None):
     """Algorithmic HBM bytes of select+plan: |Q| + |K| (bf16) + 2|S| (fp32) + |idx| + |logpi|."""
-    qk = 2 * w.B * w.H * w.N * w.d * 2
-    S = w.B * w.H * w.nQ * w.nK * 4
-    plan = w.B * w.H * w.nQ * w.s * 8
+    H = w.H if heads is None else heads
+    qk = 2 * w.B * H * w.N * w.d * 2
+    S = w.B * H * w.nQ * w.nK * 4
+    plan = w.B * H * w.nQ * w.s * 8
     return qk + 2 * S + plan
 
 
@@ -186,9 +217,10 @@ def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
-    # each rank runs an independent layer (different seed): weak scaling
-    w_r = rank_workload(w, rank)
-    Q, K, V = make_qkv(w_r, device=dev)
+    # this rank's heads of the (possibly larger) layer; inputs are drawn per global head
+    h0, h1, Ht = rank_heads(w, world, rank, args.shard)
+    Hr = h1 - h0
+    Q, K, V = make_qkv(w, device=dev, heads=range(h0, h1))
     reuse = max(1, w.plan_reuse)
     pert = []
     for c in range(reuse):
@@ -197,9 +229,10 @@ def run_ours(args, world, rank, local):
                               for k, x in enumerate((Q, K, V))))
         else:
             pert.append((Q, K, V))
-    p = ab.params(w.B, w.H, w.N, w.d, w.kv_block, w.clusters, w.kmeans_iters)
-    rows = w.B * w.H * w.nQ
-    S = torch.empty(w.B, w.H, w.nQ, w.nK, device=dev)
+    p = ab.params(w.B, Hr, w.N, w.d, w.kv_block, w.clusters, w.kmeans_iters, head0=h0,
+                  heads_total=Ht)
+    rows = w.B * Hr * w.nQ
+    S = torch.empty(w.B, Hr, w.nQ, w.nK, device=dev)
     ws = torch.empty(ab.ab_workspace_bytes(p), dtype=torch.uint8, device=dev)
     idx = torch.empty(rows, w.s, dtype=torch.int32, device=dev)
     lp = torch.empty(rows, w.s, device=dev)
@@ -270,10 +303,11 @@ def run_ours(args, world, rank, local):
     plan_ms = statistics.mean(e1.elapsed_time(e2) for e0, e1, e2, _ in ev["steps"])
     attn_ms = (statistics.mean(a0.elapsed_time(a1) for *_, att in ev["steps"] for a0, a1 in att)
                if run_attn else float("nan"))
-    F = kept_flops(w)
-    value = world * reuse * F / (ms_step * 1e-3) / 1e12
+    F = kept_flops(w, Hr)  # one attention call of this rank
+    F_all = kept_flops(w, Ht if args.shard == "strong" else w.H * world)  # all ranks
+    value = reuse * F_all / (ms_step * 1e-3) / 1e12
     attn_tflops = F / (attn_ms * 1e-3) / 1e12
-    sp_bytes = select_plan_bytes(w)
+    sp_bytes = select_plan_bytes(w, Hr)
     sp_gbs = sp_bytes / ((sel_ms + plan_ms) * 1e-3) / 1e9
 
     # select + plan overlapped across head groups on two streams (ab_select_plan), timed
@@ -297,28 +331,34 @@ def run_ours(args, world, rank, local):
     # select's exponential work at the special-function rate (16 per clock per SM)
     sm_hz = (clk.summary().get("sm_mhz") or 1800.0) * 1e6
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    sel_exp = 2 * w.clusters * w.B * w.H * w.nQ * w.nK
+    sel_exp = 2 * w.clusters * w.B * Hr * w.nQ * w.nK
     sel_sfu_ms = sel_exp / (16 * n_sms * sm_hz) * 1e3
 
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e and args.only == "all":
-        e2e = run_e2e(args, w, p, Q, K, pert, reuse, world, dev)
+        e2e = run_e2e(args, w, p, Q, K, pert, reuse, world, dev, F_all, Hr)
 
-    peak_t = peaks["bf16_tflops_sustained"]
+    peak_t = peaks["bf16_tflops"]  # burst: each attention call is timed on its own
+    peak_sus = peaks["bf16_tflops_sustained"]
+    heads_desc = (f"heads {h0}-{h1 - 1} of {Ht} on rank {rank}" if world > 1 else f"H={w.H}")
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if args.shard == "strong" else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (random-Fourier Q/K + noise, Gaussian V; seeded)",
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({'x'.join(map(str, w.latent))}) "
                                f"d={w.d} kv_block={w.kv_block} q_block=128 clusters={w.clusters} "
                                f"s={w.s}/{w.nK} plan_reuse={reuse}",
-                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
+                   "global_batch": w.B, "seq_len": w.N,
+                   "parallelism": (f"head-sharded x{world} ({'strong' if args.shard == 'strong' else 'weak'}: "
+                                   f"{Ht} heads, {heads_desc})" if world > 1 else "1 GPU"),
                    "l2": "inputs larger than L2 (Q/K/V 774 MB each), no flush"},
         "ms_per_attn_call": round(attn_ms, 3),
         "attn_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peak_t, 4),
+        "attn_frac_of_bf16_sustained_peak": round(attn_tflops / peak_sus, 4),
         "select_ms": round(sel_ms, 3), "plan_ms": round(plan_ms, 3),
         "select_plan_gbs": round(sp_gbs, 1),
         "select_plan_frac_of_hbm": round(sp_gbs / peaks["hbm_gbs"], 4),
@@ -330,9 +370,12 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "attn_kernel<128,false>",
                      "achieved": round(attn_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak_t, 4),
-                     "peak_source": f"{peaks['source']} bf16_tflops_sustained",
-                     "traffic": args.traffic if args.traffic is not None else ATTN_TRAFFIC_BYTES,
-                     "l2_gather_gbs": round(gathered_bytes(w) / (attn_ms * 1e-3) / 1e9, 1)},
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "frac_of_sustained": round(attn_tflops / peak_sus, 4),
+                     "sustained_peak": peak_sus,
+                     "traffic": attn_traffic(w, Hr),
+                     "traffic_source_sha256": attn_source_sha256()[:16],
+                     "l2_gather_gbs": round(gathered_bytes(w, Hr) / (attn_ms * 1e-3) / 1e9, 1)},
         "gpu_launches": args.steps * (4 * run_select + run_plan + reuse * run_attn),
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -342,7 +385,7 @@ def run_ours(args, world, rank, local):
     return out
 
 
-def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
+def run_e2e(args, w, p, Q, K, pert, reuse, world, dev, F_all, Hr):
     """Same step through the public API with host inputs: H2D of every input, D2H of every O."""
     import torch
 
@@ -353,8 +396,8 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
     hostO = [torch.empty(Q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(reuse)]
     dQ, dK = torch.empty_like(Q), torch.empty_like(K)
     dP = [tuple(torch.empty_like(Q) for _ in range(3)) for _ in range(reuse)]
-    rows = w.B * w.H * w.nQ
-    S = torch.empty(w.B, w.H, w.nQ, w.nK, device=dev)
+    rows = w.B * Hr * w.nQ
+    S = torch.empty(w.B, Hr, w.nQ, w.nK, device=dev)
     ws = torch.empty(ab.ab_workspace_bytes(p), dtype=torch.uint8, device=dev)
     idx = torch.empty(rows, w.s, dtype=torch.int32, device=dev)
     lp = torch.empty(rows, w.s, device=dev)
@@ -407,7 +450,7 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
 
     for i in range(2):
         step(i)
-    steps = max(1, min(args.steps, 3))
+    steps = max(1, args.steps)
     barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -421,14 +464,14 @@ def run_e2e(args, w, p, Q, K, pert, reuse, world, dev):
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
-    value = world * reuse * kept_flops(w) / (ms * 1e-3) / 1e12
+    value = reuse * F_all / (ms * 1e-3) / 1e12
     return {"value": round(value, 3), "unit": UNIT, "ms_per_step": round(ms, 2), "steps": steps,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
 def oracle_threads():
-    """Threads the oracle's numpy work runs on: the BLAS thread pool (threadpoolctl), else
-    torch's intra-op thread count."""
+    """Threads the oracle's numpy work runs on in one process: the BLAS thread pool
+    (threadpoolctl), else torch's intra-op thread count."""
     try:
         import threadpoolctl
 
@@ -443,39 +486,96 @@ def oracle_threads():
     return torch.get_num_threads()
 
 
-def cpu_baseline(w, seconds=15.0):
-    """The oracle as it stands on the host cores: select + plan + attention for a bounded
-    sample of query blocks of head 0, expressed in the metric's unit (kept-block FLOP/s)."""
-    import numpy as np
+# ---- the oracle on all host cores: one worker process per core, one BLAS thread each.
+# Workers start with "spawn" (a process forked after CUDA was initialised can hang) and
+# each draws head 0 of the workload and pools its keys once, before the timed region.
 
-    from block_sparse_attention_ibcs_b200.inputs import make_qkv
+_OB = {}
+
+
+def _oracle_worker_init(name):
+    import threadpoolctl
+
+    from block_sparse_attention_ibcs_b200.inputs import WORKLOADS, make_qkv
     from oracle import abattn_oracle as O
 
+    threadpoolctl.threadpool_limits(1)
+    w = WORKLOADS[name]
     Q, K, V = make_qkv(w, device="cpu", heads=[0])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
-    cores = oracle_threads()
     t0 = time.perf_counter()
     Kp = O.pool_keys(k, w.kv_block)
-    done = 0
-    rows_done = 0
-    qbs = np.random.default_rng(0).permutation(w.nQ)  # fixed order; stops at the time budget
-    for i in qbs:
-        i = int(i)
-        Qb = q[i * 128: min(w.N, (i + 1) * 128)]
-        cent, wt, _, _ = O.kmeans_block(Qb, w.clusters, w.kmeans_iters)
-        S = O.block_scores(cent, wt, Kp).astype(np.float32)
-        idx, lp, _ = O.plan_row(S, w.s, w.philox_seed, 0, i)
-        O.attn_block(Qb, k, v, idx, lp, w.kv_block)
-        done += 1
-        rows_done += Qb.shape[0]
-        if time.perf_counter() - t0 > seconds:
-            break
-    dt = time.perf_counter() - t0
-    flops = 4.0 * rows_done * (w.s * w.kv_block) * w.d
-    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"head 0, {done} query blocks (select+plan+attn per block, pooling of the "
-                      f"whole head included), {dt:.1f} s",
-            "ms_per_query_block": round(1e3 * dt / done, 1)}
+    _OB.update(w=w, q=q, k=k, v=v, Kp=Kp, pool_s=time.perf_counter() - t0)
+
+
+def _oracle_worker_ping(_):
+    time.sleep(0.2)
+    return _OB["pool_s"]
+
+
+def _oracle_query_block(i):
+    """Select + plan + attention of query block i of head 0; returns its valid rows."""
+    from oracle import abattn_oracle as O
+
+    w, q, k, v, Kp = _OB["w"], _OB["q"], _OB["k"], _OB["v"], _OB["Kp"]
+    Qb = q[i * 128: min(w.N, (i + 1) * 128)]
+    cent, wt, _, _ = O.kmeans_block(Qb, w.clusters, w.kmeans_iters)
+    S = O.block_scores(cent, wt, Kp).astype(np.float32)
+    idx, lp, _ = O.plan_row(S, w.s, w.philox_seed, 0, i)
+    O.attn_block(Qb, k, v, idx, lp, w.kv_block)
+    return Qb.shape[0]
+
+
+class OraclePool:
+    """The oracle as it stands, parallel over query blocks on the host's cores."""
+
+    def __init__(self, w, procs=None):
+        import multiprocessing as mp
+
+        self.w = w
+        self.procs = procs or os.cpu_count() or 1
+        self.pool = mp.get_context("spawn").Pool(self.procs, _oracle_worker_init, (w.name,))
+        # every worker has drawn its inputs and pooled the keys before anything is timed
+        pings = self.pool.map(_oracle_worker_ping, range(2 * self.procs), chunksize=1)
+        self.pool_s = max(pings)
+        self.order = [int(i) for i in np.random.default_rng(0).permutation(w.nQ)]
+        self.next = 0
+
+    def run(self, seconds):
+        """Query blocks in a fixed order until about `seconds` of wall time have passed;
+        returns (kept-block FLOP/s, description).  The head's key pooling, done once per
+        worker, is charged in proportion to the query blocks processed."""
+        w = self.w
+        t0 = time.perf_counter()
+        rows = done = 0
+        while time.perf_counter() - t0 < seconds:
+            batch = [self.order[(self.next + k) % w.nQ] for k in range(self.procs)]
+            self.next += self.procs
+            for r in self.pool.map(_oracle_query_block, batch, chunksize=1):
+                rows += r
+                done += 1
+        dt = time.perf_counter() - t0 + self.pool_s * done / w.nQ
+        flops = 4.0 * rows * (w.s * w.kv_block) * w.d
+        sample = (f"head 0, {done} query blocks (k-means, scores, plan, attention per block; the "
+                  f"head's key pooling charged pro rata), {self.procs} processes x 1 BLAS thread, "
+                  f"{dt:.1f} s")
+        return flops / dt, sample, 1e3 * dt * self.procs / done
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline(w, seconds=15.0):
+    """The oracle as it stands on all host cores (one process per core) for a bounded
+    sample of query blocks of head 0, in the metric's unit (kept-block FLOP/s)."""
+    pool = OraclePool(w)
+    try:
+        v, sample, ms_qb = pool.run(seconds)
+    finally:
+        pool.close()
+    return {"value": round(v / 1e12, 6), "unit": UNIT, "cores": pool.procs, "kind": "oracle",
+            "sample": sample, "ms_per_query_block_per_core": round(ms_qb, 1)}
 
 
 def run_sweep(args):
@@ -552,12 +652,16 @@ def run_reference(args, world, rank):
     from block_sparse_attention_ibcs_b200.inputs import WORKLOADS
 
     w = WORKLOADS[args.workload]
-    per = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    per = getattr(args, "ref_seconds", None) or max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     vals = []
-    for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(w, seconds=per)
-        if i >= args.warmup:
-            vals.append(cb)
+    pool = OraclePool(w)
+    try:
+        for i in range(args.warmup + args.steps):
+            v, sample, _ = pool.run(per)
+            if i >= args.warmup:
+                vals.append({"value": v / 1e12, "sample": sample})
+    finally:
+        pool.close()
     value = statistics.mean(c["value"] for c in vals)
     ms_step = 1e3 * 4.0 * w.B * w.H * w.N * (w.s * w.kv_block) * w.d * max(1, w.plan_reuse) / (value * 1e12)
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -566,7 +670,7 @@ def run_reference(args, world, rank):
             "data": "synthetic (seeded)",
             "config": {"workload": f"{w.name} (bounded sample per step, extrapolated)",
                        "global_batch": w.B, "seq_len": w.N, "parallelism": "cpu"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"],
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs,
                              "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -585,8 +689,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per attention launch from an ncu capture of this kernel")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="reference arm: seconds of oracle work per step (default: 60 s over all steps)")
+    ap.add_argument("--shard", default="weak", choices=["weak", "strong"],
+                    help="N>1: a layer of H*N heads, H per rank (weak), or the layer's H heads "
+                         "split over the ranks (strong)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -19,7 +19,7 @@ import os
 __all__ = [
     "ABError", "ABParams", "params", "lib", "ab_workspace_bytes", "ab_select",
     "ab_select_debug", "ab_select_plan", "ab_plan", "ab_plan_variant", "ab_sample", "ab_attn",
-    "ab_attn_dense",
+    "ab_attn_dense", "ab_attn_debug", "ab_select_noalloc",
     "ab_get_status", "ab_status_string", "ab_version", "LIB_PATH", "PLAN_MODES",
 ]
 
@@ -43,11 +43,15 @@ class ABError(RuntimeError):
 
 class ABParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("B", "H", "N", "d", "q_block", "kv_block", "clusters", "kmeans_iters")]
+                ("B", "H", "N", "d", "q_block", "kv_block", "clusters", "kmeans_iters", "head0",
+                 "heads_total")]
 
 
-def params(B, H, N, d, kv_block=4, clusters=8, kmeans_iters=1, q_block=128) -> ABParams:
-    return ABParams(B, H, N, d, q_block, kv_block, clusters, kmeans_iters)
+def params(B, H, N, d, kv_block=4, clusters=8, kmeans_iters=1, q_block=128, head0=0,
+           heads_total=0) -> ABParams:
+    """Parameters of a call over heads [head0, head0 + H) of a layer of heads_total heads
+    (heads_total = 0: the call is the whole layer)."""
+    return ABParams(B, H, N, d, q_block, kv_block, clusters, kmeans_iters, head0, heads_total)
 
 
 _LIB = None

@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include <cudaTypedefs.h>
 
 #include "abattn.h"
@@ -29,6 +31,7 @@ int ilog2_exact(int v) {
 
 struct Dims {
   int B, H, N, d, bk, C, iters;
+  int h0, Ht;  // this call's heads are [h0, h0 + H) of a layer of Ht heads
   long long BH, nQ, nK;
 };
 
@@ -40,15 +43,23 @@ ab_status check_params(const ab_params* p, Dims* out) {
   if (p->q_block != 128) return AB_ERR_UNSUPPORTED;
   if (p->d != 64 && p->d != 128) return AB_ERR_UNSUPPORTED;
   if (p->clusters > CMAX || p->kmeans_iters > 4) return AB_ERR_UNSUPPORTED;
+  if (p->head0 < 0 || p->heads_total < 0) return AB_ERR_INVALID_ARG;
+  if (p->heads_total == 0 ? p->head0 != 0 : (long long)p->head0 + p->H > p->heads_total)
+    return AB_ERR_INVALID_ARG;
   Dims d;
   d.B = p->B; d.H = p->H; d.N = p->N; d.d = p->d; d.bk = p->kv_block;
   d.C = p->clusters; d.iters = p->kmeans_iters;
+  d.h0 = p->head0;
+  d.Ht = p->heads_total > 0 ? p->heads_total : p->H;
   d.BH = (long long)p->B * p->H;
   d.nQ = (p->N + 127) / 128;
   d.nK = (p->N + p->kv_block - 1) / p->kv_block;
   // grid and index limits: every (b,h,query block) is one CTA of a 1-D grid and
-  // element offsets must fit the kernels' size_t arithmetic; nK*2^32 must fit uint64
-  if (d.BH * d.nQ > 0x7fffffffLL || d.nK > (1LL << 30)) return AB_ERR_UNSUPPORTED;
+  // element offsets must fit the kernels' size_t arithmetic; nK*2^32 must fit uint64; the
+  // whole layer's plan rows number the 32-bit Philox counter word
+  if (d.BH * d.nQ > 0x7fffffffLL || (long long)d.B * d.Ht * d.nQ > 0x7fffffffLL ||
+      d.nK > (1LL << 30))
+    return AB_ERR_UNSUPPORTED;
   *out = d;
   return AB_OK;
 }
@@ -79,6 +90,21 @@ Workspace carve(const Dims& d, void* base) {
   return ws;
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+int device_sms() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 ab_status launch_status() {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -102,6 +128,29 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Unique id of the calling thread's current CUDA context (ids are never reused within a
+// process, unlike context handles), through the driver entry points the runtime exposes.
+// Per-device host caches of device objects key on it, so that a cache filled in a context
+// that was destroyed since (cudaDeviceReset) is refilled instead of used.
+bool current_context_id(unsigned long long* id) {
+  static const auto fns = [] {
+    void* get = nullptr;
+    void* getid = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &get, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      get = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &getid, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      getid = nullptr;
+    return std::make_pair((PFN_cuCtxGetCurrent_v4000)get, (PFN_cuCtxGetId_v12000)getid);
+  }();
+  if (!fns.first || !fns.second) return false;
+  CUcontext ctx = nullptr;
+  if (fns.first(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return fns.second(ctx, id) == CUDA_SUCCESS;
+}
+
 // Tensor map of a bf16 array [z][y][x] (x contiguous, x = d elements) read in boxes of
 // 64 x box_y x 1 with the 128-byte swizzle; out-of-range rows read as zeros.
 bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z, uint32_t box_y) {
@@ -116,11 +165,11 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// split_bh: the head count the score passes' work split is chosen for (the whole tensor's,
-// also when this launch covers a slice of its heads)
+// The score passes' work split is chosen for the whole layer's B * Ht heads, also when this
+// launch covers a slice of them.
 template <int D>
 ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, const Workspace& ws,
-                     int8_t* labels, cudaStream_t st, long long split_bh = 0) {
+                     int8_t* labels, cudaStream_t st) {
   SelectArgs a;
   a.Q = (const uint16_t*)Q;
   a.K = (const uint16_t*)K;
@@ -138,11 +187,13 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
   a.C = d.C;
   a.iters = d.iters;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  const int sms = device_sms();
   const size_t units = (size_t)d.BH * d.nK * (D / 8);
-  const int pool_blocks = (int)((units + 255) / 256 < 148 * 32 ? (units + 255) / 256 : 148 * 32);
+  const size_t pool_cap = (size_t)sms * 32;
+  const int pool_blocks = (int)((units + 255) / 256 < pool_cap ? (units + 255) / 256 : pool_cap);
   pool_kernel<D><<<pool_blocks, 256, 0, st>>>(a);
   kmeans_kernel<D><<<(unsigned)(d.BH * d.nQ), KM_THREADS, 0, st>>>(a);
-  const ScoreSplit sp = score_split(d.BH, d.nQ, d.nK, split_bh > 0 ? split_bh : d.BH);
+  const ScoreSplit sp = score_split(d.BH, d.nQ, d.nK, (long long)d.B * d.Ht, sms);
   using SL = ScoreSmem<D>;
   if (cudaFuncSetAttribute(score_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SL::ALLOC) != cudaSuccess ||
@@ -160,10 +211,16 @@ ab_status run_select(const Dims& d, const void* Q, const void* K, float* S, cons
   return launch_status();
 }
 
+// bh0: flattened (b, h) index of this launch's first head within the call (a launch over a
+// slice of the call's heads, as ab_select_plan makes)
 ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t offset,
-                   int mode, int32_t* idx, float* logpi, cudaStream_t st, long long row0 = 0) {
+                   int mode, int32_t* idx, float* logpi, cudaStream_t st, long long bh0 = 0) {
   PlanArgs a;
-  a.row0 = (int)row0;
+  a.nQ = (int)d.nQ;
+  a.H = d.H;
+  a.Ht = d.Ht;
+  a.h0 = d.h0;
+  a.bh0 = bh0;
   a.S = S;
   a.idx = idx;
   a.logpi = logpi;
@@ -316,16 +373,15 @@ ab_status select_plan_slice(const Dims& d, long long bh0, long long n, const voi
   const void* Kg = (const uint16_t*)K + qk;
   float* Sg = S + (size_t)bh0 * d.nQ * d.nK;
   Workspace wsp = carve(g, ws);
-  ab_status r = (d.d == 128) ? run_select<128>(g, Qg, Kg, Sg, wsp, nullptr, st_sel, d.BH)
-                             : run_select<64>(g, Qg, Kg, Sg, wsp, nullptr, st_sel, d.BH);
+  ab_status r = (d.d == 128) ? run_select<128>(g, Qg, Kg, Sg, wsp, nullptr, st_sel)
+                             : run_select<64>(g, Qg, Kg, Sg, wsp, nullptr, st_sel);
   if (r != AB_OK) return r;
   if (st_plan != st_sel) {
     if (cudaEventRecord(ev, st_sel) != cudaSuccess || cudaStreamWaitEvent(st_plan, ev, 0) != cudaSuccess)
       return launch_status();
   }
   const size_t rows = (size_t)bh0 * d.nQ;
-  return run_plan(g, Sg, s, seed, offset, AB_PLAN_SIP, idx + rows * s, logpi + rows * s, st_plan,
-                  (long long)rows);
+  return run_plan(g, Sg, s, seed, offset, AB_PLAN_SIP, idx + rows * s, logpi + rows * s, st_plan, bh0);
 }
 
 }  // namespace
@@ -357,6 +413,56 @@ ab_status ab_plan(const ab_params* p, const float* S, int s, uint64_t seed, uint
   return plan_common(p, S, s, seed, offset, AB_PLAN_SIP, idx, logpi, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// ab_select_plan's events (one per head group plus one for the end): created once per
+// device context and reused by every call.  The mutex serialises the calls' enqueue
+// sequences, so one call's records and waits never interleave with another host thread's.
+constexpr int kSpMaxGroups = 64;
+std::mutex g_sp_mu;
+struct SpEvents {
+  unsigned long long ctx = 0;
+  bool made = false;
+  cudaEvent_t ev[kSpMaxGroups + 1];
+};
+SpEvents g_sp_events[64];
+
+// Events of the current device's context; call with g_sp_mu held.
+ab_status select_plan_events(cudaEvent_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status();
+  if (dev < 0 || dev >= 64) return AB_ERR_UNSUPPORTED;
+  SpEvents& e = g_sp_events[dev];
+  unsigned long long ctx = 0;
+  if (e.made && current_context_id(&ctx) && e.ctx == ctx) {
+    *out = e.ev;
+    return AB_OK;
+  }
+  // first call in this context (the events of a context destroyed since are dropped); creating
+  // an event also creates the device's context if there is none yet
+  e.made = false;
+  for (int g = 0; g <= kSpMaxGroups; ++g)
+    if (cudaEventCreateWithFlags(&e.ev[g], cudaEventDisableTiming) != cudaSuccess) {
+      for (int k = 0; k < g; ++k) cudaEventDestroy(e.ev[k]);
+      return launch_status();
+    }
+  if (!current_context_id(&ctx)) {
+    for (int g = 0; g <= kSpMaxGroups; ++g) cudaEventDestroy(e.ev[g]);
+    fprintf(stderr, "abattn: cannot identify the current CUDA context\n");
+    return AB_ERR_CUDA;
+  }
+  e.made = true;
+  e.ctx = ctx;
+  *out = e.ev;
+  return AB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 ab_status ab_select_plan(const ab_params* p, const void* Q, const void* K, float* S, void* ws,
                          size_t ws_bytes, int s, uint64_t seed, uint64_t offset, int32_t* idx,
                          float* logpi, int groups, void* stream, void* stream2) {
@@ -375,15 +481,14 @@ ab_status ab_select_plan(const ab_params* p, const void* Q, const void* K, float
   // compute-bound and their CTAs do not fit on one SM together (shared memory).
   long long G = groups > 0 ? groups : 1;
   if (G > d.BH) G = d.BH;
-  // events: one per group (select of group g done -> plan of group g may start), one for the end
-  cudaEvent_t evs[65];
-  if (G > 64) G = 64;
-  for (long long g = 0; g <= G; ++g)
-    if (cudaEventCreateWithFlags(&evs[g], cudaEventDisableTiming) != cudaSuccess) {
-      for (long long k = 0; k < g; ++k) cudaEventDestroy(evs[k]);
-      return launch_status();
-    }
-  r = AB_OK;
+  if (G > kSpMaxGroups) G = kSpMaxGroups;
+  // events: one per group (select of group g done -> plan of group g may start), one for the
+  // end.  A wait refers to the record enqueued last before it, so reusing the events across
+  // calls is safe while the enqueue sequences do not interleave (the mutex).
+  std::lock_guard<std::mutex> lock(g_sp_mu);
+  cudaEvent_t* evs = nullptr;
+  r = select_plan_events(&evs);
+  if (r != AB_OK) return r;
   for (long long g = 0; g < G && r == AB_OK; ++g) {
     const long long b0 = d.BH * g / G, b1 = d.BH * (g + 1) / G;
     r = select_plan_slice(d, b0, b1 - b0, Q, K, S, ws, s, seed, offset, idx, logpi, sa, sb, evs[g]);
@@ -391,7 +496,6 @@ ab_status ab_select_plan(const ab_params* p, const void* Q, const void* K, float
   // the caller's stream sees every plan as done
   if (r == AB_OK && (cudaEventRecord(evs[G], sb) != cudaSuccess || cudaStreamWaitEvent(sa, evs[G], 0) != cudaSuccess))
     r = launch_status();
-  for (long long g = 0; g <= G; ++g) cudaEventDestroy(evs[g]);  // released once their work is done
   return r;
 }
 
@@ -464,8 +568,6 @@ int ab_version(void) { return 100; }
 // below instead of a caller buffer.
 // ------------------------------------------------------------------------------------
 
-#include <mutex>
-
 // Capacity of the built-in scratch.  Every GPU that loads the library holds this much
 // device memory until the process exits.
 #define AB_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -477,25 +579,36 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  The host-side symbol is
 // only a stand-in, so the address is looked up once per device (with that device
-// current) and cached.
+// current) and cached together with the id of the context it belongs to; a call in a
+// newer context of the device (after cudaDeviceReset, the old address is gone) looks it
+// up again.
 ab_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return launch_status();
   if (dev < 0 || dev >= kMaxDevices) return AB_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (g_noalloc_addr[dev] == nullptr || !have_ctx || g_noalloc_ctx[dev] != ctx) {
     void* addr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&addr, g_ab_noalloc_scratch);
     if (e != cudaSuccess || addr == nullptr) {
       fprintf(stderr, "abattn: cannot resolve the built-in scratch on device %d: %s\n", dev,
               cudaGetErrorString(e));
       cudaGetLastError();
+      g_noalloc_addr[dev] = nullptr;
       return AB_ERR_CUDA;
     }
-    g_noalloc_addr[dev] = addr;
+    // the lookup made the context current if it was not; cache under its id
+    const bool have_now = have_ctx || current_context_id(&ctx);
+    g_noalloc_addr[dev] = have_now ? addr : nullptr;  // no id: look up again next call
+    g_noalloc_ctx[dev] = ctx;
+    *out = addr;
+    return AB_OK;
   }
   *out = g_noalloc_addr[dev];
   return AB_OK;

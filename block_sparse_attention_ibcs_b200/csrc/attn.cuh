@@ -75,7 +75,7 @@ struct AttnArgs {
 // Event tracing (TRACE builds only): CTAs 0, 1 and the one at a third of the grid record
 // clock64() per tile for the events below into trace[((slot * 16) + event) * 128 + t].
 enum { EV_COPY_START = 0, EV_COPY_ISSUED, EV_SM_LOADED, EV_SM_MAX, EV_LANDED, EV_QK,
-       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_SM_SFULL,
+       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_UNUSED12,
        EV_SM_PDONE_W1, EV_SM_PDONE_W2, EV_SM_PDONE_W3, EV_COUNT };
 constexpr int TRACE_TILES = 128;
 
@@ -194,13 +194,31 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         lr[k] = in ? __ldg(a.logpi + plan_off + m) : 0.f;
       }
     };
-    auto check = [&](int (&jr)[4]) {
+    // An entry is used only if it lies in [0, nK) and is above every earlier entry of its
+    // row (plans are strictly ascending, so no block can count twice); any other entry is
+    // masked (-1: its rows become padding) and flags AB_ERR_DEVICE_CHECK.  The earlier
+    // entries' maximum comes from a max-scan over the lanes and the running maximum of the
+    // row's previous tiles (row_max), so the check holds across tile edges.
+    int row_max = INT_MIN;
+    auto check = [&](int t, int (&jr)[4]) {
       bool bad = false;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const bool ok = jr[k] >= 0 && jr[k] < a.nK;
-        bad |= (jr[k] != PAD) && !ok;
-        jr[k] = ok ? jr[k] : -1;
+        if (32 * k >= nb) break;  // warp-uniform: registers past the tile's blocks hold padding
+        const int e = lane + 32 * k;
+        const bool in = e < nb && t * nb + e < a.s;
+        int incl = in ? jr[k] : INT_MIN;  // inclusive max over lanes 0..lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl = max(incl, y);
+        }
+        int before = __shfl_up_sync(0xffffffffu, incl, 1);
+        before = max(row_max, lane == 0 ? INT_MIN : before);  // max of the earlier entries
+        const bool ok = jr[k] >= 0 && jr[k] < a.nK && jr[k] > before;
+        bad |= in && !ok;
+        jr[k] = (in && ok) ? jr[k] : (in ? -1 : PAD);
+        row_max = max(row_max, __shfl_sync(0xffffffffu, incl, 31));
       }
       if (bad) ab_flag(AB_ERR_DEVICE_CHECK);
     };
@@ -221,7 +239,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     };
     if (!DENSE) {
       fetch(0, jc, lc);
-      check(jc);
+      check(0, jc);
     }
 
     int st = 0;  // t % ATTN_STAGES
@@ -300,7 +318,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           jc[k] = jn[k];
           lc[k] = ln[k];
         }
-        check(jc);
+        check(t + 1, jc);
       }
       st = (st + 1 == ATTN_STAGES) ? 0 : st + 1;
       if (p == 0) ev(EV_COPY_ISSUED, t);

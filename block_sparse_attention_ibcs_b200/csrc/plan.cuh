@@ -50,10 +50,21 @@ struct PlanArgs {
   int nK, s;
   uint64_t seed, offset;
   int mode;         // ab_plan_mode: SIP, SIP without inverse-probability weights, uniform
-  int row0;         // row index of this launch's first row in the whole (b, h, i) order
-                    // (the Philox counter uses it: a launch over a slice of heads draws as
-                    // the full launch would)
+  // Philox row numbering.  Launch row r is query block r % nQ of (b, h) = the flattened
+  // head bh0 + r / nQ of the call (B x H heads); the draw uses that row's index in the
+  // whole layer, (b * Ht + h0 + h) * nQ + i, so a launch over a slice of the call, or a
+  // call over a slice of a layer's heads, draws exactly as one launch over the layer.
+  int nQ, H, Ht, h0;
+  long long bh0;
 };
+
+// Counter word of launch row r (fits 32 bits: the host checks B * Ht * nQ < 2^31).
+AB_DEV uint32_t plan_counter_row(const PlanArgs& a, int r) {
+  const long long bl = a.bh0 + r / a.nQ;
+  const int i = r - (r / a.nQ) * a.nQ;
+  const long long b = bl / a.H, h = bl - b * a.H;
+  return (uint32_t)((b * a.Ht + a.h0 + h) * a.nQ + i);
+}
 
 // Philox4x32-10 (Salmon et al., SC'11), word 0 of the output block.
 AB_DEV uint32_t philox4x32_10_w0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
@@ -505,7 +516,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   uint64_t sat_before, rest_before, n_sat, tot_rest;
   block_exscan2_1b(my_sat, my_rest, ru, par, sat_before, rest_before, n_sat, tot_rest);
 
-  const uint32_t U = philox4x32_10_w0((uint32_t)(a.row0 + row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
+  const uint32_t U = philox4x32_10_w0(plan_counter_row(a, row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
                                       0u, (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
   // lattice points U + k 2^32 below x, for 0 <= x <= s 2^32 (U < 2^32)
   const uint64_t CB = TWO32 - 1u - (uint64_t)U;

@@ -9,7 +9,9 @@
 //
 // Exactness: pooled keys and centroids are rounded once to bf16 from fp64 means (sums
 // of at most 128 bf16 values are exact in fp64, the division is IEEE), so they equal
-// the CPU reference bit for bit; assignments use fp64 distances.  Logits use the bf16
+// the CPU reference bit for bit.  Assignments are decided in fp32 with a certified error
+// margin; a row whose best and second-best distances are closer than that margin is
+// decided again in fp64, so the labels equal the exact argmin.  Logits use the bf16
 // operands with fp32 accumulation; softmax statistics are fp32 in the log2 domain.
 //
 //   pool_kernel      Kp[bh, j, :]  = bf16(mean of block j's valid keys)
@@ -340,7 +342,10 @@ constexpr int SC_MMA_WARP = 17;            // TMEM allocation, MMA issue
 constexpr int SC_THREADS = SC_CONSUMERS + 64;
 constexpr int SC_STAGES = 3;
 constexpr int SC_MAX_CHUNKS = 8;           // key chunks per group (pass-1 partial slots)
-constexpr int SC_GRID = 148;               // CTAs: one per B200 SM
+// The chunk count is chosen for a fixed nominal grid of 148 CTAs (B200's SM count), not
+// for the device at hand: chunk boundaries decide how S is rounded, so S stays the same
+// on every device.  The launch itself uses one CTA per SM of the device.
+constexpr int SC_SPLIT_GRID = 148;
 constexpr float SC_LAZY_LIMIT = 1048576.f;  // 2^20
 
 template <int D>
@@ -373,15 +378,17 @@ struct ScoreSplit {
   int CT;       // tiles per chunk
   int KC;       // chunks per group: ceil(T / CT) <= SC_MAX_CHUNKS
   long long U;  // units = B*H * G * KC
-  int P;        // CTAs = min(U, SC_GRID)
+  int P;        // CTAs = min(U, SMs of the device)
 };
 
 // The number of key chunks per group trades load balance (more, shorter units) against
 // the centroid reload at every unit (measured on B200 at about two tiles of time): choose
 // the count that minimises (units of the busiest CTA) x (tiles per unit + 2) for a tensor
-// of BH_choice heads.  A launch over a slice of heads passes the whole tensor's head count,
-// so its chunks -- and with them the rounding of S -- are those of the whole launch.
-inline ScoreSplit score_split(long long BH, long long nQ, long long nK, long long BH_choice) {
+// of BH_choice heads on the nominal grid.  A launch over a slice of heads passes the whole
+// layer's head count, so its chunks -- and with them the rounding of S -- are those of one
+// launch over the whole layer.
+inline ScoreSplit score_split(long long BH, long long nQ, long long nK, long long BH_choice,
+                              int sms) {
   ScoreSplit s;
   s.G = (int)((nQ + SC_QB - 1) / SC_QB);
   s.T = (int)((nK + 127) / 128);
@@ -390,7 +397,7 @@ inline ScoreSplit score_split(long long BH, long long nQ, long long nK, long lon
   for (int k = 1; k <= SC_MAX_CHUNKS && k <= s.T; ++k) {
     const int ct = (s.T + k - 1) / k;
     const int kc = (s.T + ct - 1) / ct;
-    const long long per_cta = (R * kc + SC_GRID - 1) / SC_GRID;
+    const long long per_cta = (R * kc + SC_SPLIT_GRID - 1) / SC_SPLIT_GRID;
     const long long cost = per_cta * (ct + 2);
     if (best < 0 || cost < best) {
       best = cost;
@@ -399,7 +406,7 @@ inline ScoreSplit score_split(long long BH, long long nQ, long long nK, long lon
     }
   }
   s.U = BH * s.G * s.KC;
-  s.P = (int)(s.U < SC_GRID ? s.U : SC_GRID);
+  s.P = (int)(s.U < sms ? s.U : sms);
   return s;
 }
 

@@ -55,18 +55,33 @@ typedef enum {
  *   kv_block      KV block: a power of two in [1, 128]; the page uses 4
  *   clusters      query clusters per query block, 1..8; the page uses 8
  *   kmeans_iters  Lloyd iterations after the segment-mean start, 0..4; the page uses 1
- *                 (0 = the position-based 16-query segment means of the ablation)     */
+ *                 (0 = the position-based 16-query segment means of the ablation)
+ *   head0, heads_total
+ *                 head sharding (no counterpart on the page, which runs on one GPU):
+ *                 this call covers heads [head0, head0 + H) of a layer of heads_total
+ *                 heads.  heads_total = 0 means the call is the whole layer (head0 must
+ *                 then be 0); otherwise 0 <= head0 and head0 + H <= heads_total.  Every
+ *                 tensor argument holds only this call's heads ([B, H, ...]).  Each head
+ *                 is computed independently, and the two places where the whole layer
+ *                 matters use the whole layer's numbering: the planner's Philox row is
+ *                 (b * heads_total + head0 + h) * nQ + i, and the selector cuts its
+ *                 work (and so rounds S) as for B * heads_total heads.  So S, idx, logpi
+ *                 and O of a slice are bitwise equal to the matching rows of one call
+ *                 over the whole layer.  A zero-initialised struct is the whole layer.  */
 typedef struct {
   int B, H, N, d;
   int q_block;
   int kv_block;
   int clusters;
   int kmeans_iters;
+  int head0;
+  int heads_total;
 } ab_params;
 
 /* Bytes of device workspace ab_select needs for `p` (pooled keys, centroids, shares and
  * per-centroid softmax statistics).  Writes *bytes; returns AB_ERR_INVALID_ARG /
- * AB_ERR_UNSUPPORTED for bad parameters.                                              */
+ * AB_ERR_UNSUPPORTED for bad parameters.  Only the selector takes a workspace: the
+ * planner and the attention kernel keep their working state on chip.                */
 ab_status ab_workspace_bytes(const ab_params* p, size_t* bytes);
 
 /* IBCS block scores ("how it differs" section of the AB-Attention page).
@@ -96,7 +111,8 @@ ab_status ab_select_debug(const ab_params* p, const void* Q, const void* K, floa
  * 2^-32 fixed point (lambda = the smallest fp32 whose fixed-point sum reaches s; the
  * last non-saturated blocks are trimmed so the sum is exactly s), then systematic
  * sampling of exactly s distinct blocks with one Philox4x32-10 draw
- * (key = seed, counter = (row, offset_lo, offset_hi, 0), row = (b*H + h)*nQ + i).
+ * (key = seed, counter = (row, offset_lo, offset_hi, 0), row = (b*H + h)*nQ + i for a
+ * whole layer, (b*heads_total + head0 + h)*nQ + i for a head slice).
  * Blocks with pi = 1 are always sampled.  If fewer than s blocks have S > 0, all of
  * them and the lowest-index zero blocks are taken with pi = 1.
  *   S      fp32 [B,H,nQ,nK] (device, read); entries <= 0 or NaN count as 0
@@ -157,8 +173,10 @@ ab_status ab_plan_variant(const ab_params* p, const float* S, int s, uint64_t se
  *   z_t = q.k_t / sqrt(d) - logpi_j,
  * computed in one online-softmax pass over ceil(s*kv_block/128) tiles of 128 gathered
  * tokens (tcgen05 MMAs, fp32 accumulation in tensor memory, O rounded to bf16).
- *   idx, logpi  as produced by ab_plan: int32/fp32 [B,H,nQ,s]; idx entries must lie in
- *               [0, nK) (others are masked out and flag AB_ERR_DEVICE_CHECK)
+ *   idx, logpi  as produced by ab_plan: int32/fp32 [B,H,nQ,s]; each row's idx entries
+ *               must lie in [0, nK) and be strictly ascending (so no block counts
+ *               twice).  An entry that breaks either rule is masked out (its block gets
+ *               weight 0) and the status word records AB_ERR_DEVICE_CHECK.
  *   O           bf16 [B,H,N,d] (device, written)                                      */
 ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* V,
                   const int32_t* idx, const float* logpi, int s, void* O, void* stream);
@@ -176,9 +194,14 @@ ab_status ab_attn_dense(const ab_params* p, const void* Q, const void* K, const 
  *  - trace (device, may be NULL; 8-byte aligned, 3*16*128 uint64, zeroed by the caller):
  *    a separately compiled traced kernel records clock64() for each pipeline event of
  *    tiles 0..127 of CTAs 0, 1 and gridDim/3, at trace[(slot*16 + event)*128 + tile];
- *    events: 0 K copy issued, 1 K arrival, 2 V copy issued, 3 V arrival, 4 K landed (seen
- *    by the MMA warp), 5 QK issued, 6 V landed, 7 PV issued, 8 softmax tile start,
- *    9 S ready, 10 P written, 11 CTA end (tile slot 0).
+ *    events (producer warps: 0, 1; MMA warp: 4, 5, 7; softmax warps: the rest):
+ *      0 the tile's copies start (its ring stage is free)   1 all its copies are issued
+ *      2 S loaded from tensor memory                         3 exponentials done (P built)
+ *      4 K rows and shifts landed (seen by the MMA warp)     5 QK MMAs issued
+ *      6 the P buffer is free (PV two tiles back done)       7 PV MMAs issued
+ *      8 softmax tile start                                  9 S ready (QK done)
+ *      10 P stored by warp 0                                 11 CTA end (tile slot 0)
+ *      12 unused                                             13, 14, 15 P stored by warps 1, 2, 3
  * With skip_first_arrival = 0 and trace = NULL it is ab_attn with another wait limit.   */
 ab_status ab_attn_debug(const ab_params* p, const void* Q, const void* K, const void* V,
                         const int32_t* idx, const float* logpi, int s, void* O,
@@ -209,7 +232,9 @@ int ab_version(void);
  * N = 75,600 at d = 128) are rejected with AB_ERR_WORKSPACE and a message on stderr;
  * use ab_select for them.
  *  - The first call on each device looks up the array's device address (with that device
- *    current) and caches it; make that first call before any stream capture.
+ *    current) and caches it for the device's current CUDA context; make that first call
+ *    before any stream capture.  A call in a new context of the device (after
+ *    cudaDeviceReset, say) looks the address up again.
  *  - All calls on a device share the one array and it keeps the previous call's contents
  *    (every byte the selector reads is written earlier in the same call, so nothing has
  *    to be cleared).  Calls whose work overlaps on the GPU -- on different streams, or

@@ -54,14 +54,26 @@ def test_workspace_bytes():
     (dict(B=0), -1), (dict(H=0), -1), (dict(B=-3), -1),
     # size limits: (b, h, query block) CTAs must fit a 1-D grid, nK * 2^32 a uint64
     (dict(B=1, H=4_000_000, N=75600), -2), (dict(N=(1 << 31) - 1, kv_block=1), -2),
+    # head slices: [head0, head0 + H) must lie inside the layer's heads_total heads
+    (dict(head0=1), -1), (dict(head0=-1, heads_total=8), -1), (dict(heads_total=-2), -1),
+    (dict(head0=7, heads_total=8), -1), (dict(head0=0, heads_total=1), -1),
+    # the whole layer's plan rows must fit the 32-bit Philox counter word
+    (dict(N=75600, heads_total=4_000_000), -2),
 ])
 def test_bad_params_rejected(bad, code):
-    kw = dict(B=1, H=2, N=1024, d=64, kv_block=4, clusters=8, kmeans_iters=1, q_block=128)
+    kw = dict(B=1, H=2, N=1024, d=64, kv_block=4, clusters=8, kmeans_iters=1, q_block=128,
+              head0=0, heads_total=0)
     kw.update(bad)
     p = ab.ABParams(kw["B"], kw["H"], kw["N"], kw["d"], kw["q_block"], kw["kv_block"],
-                    kw["clusters"], kw["kmeans_iters"])
+                    kw["clusters"], kw["kmeans_iters"], kw["head0"], kw["heads_total"])
     n = ctypes.c_size_t(0)
     assert ab.lib().ab_workspace_bytes(ctypes.byref(p), ctypes.byref(n)) == code
+
+
+@pytest.mark.parametrize("head0,heads_total", [(0, 0), (0, 2), (6, 8), (3, 40)])
+def test_head_slices_accepted(head0, heads_total):
+    p = ab.params(1, 2, 1024, 64, head0=head0, heads_total=heads_total)
+    assert ab.ab_workspace_bytes(p) == ab.ab_workspace_bytes(ab.params(1, 2, 1024, 64))
 
 
 def test_largest_accepted_grid():

@@ -6,7 +6,7 @@ import bench
 
 
 def test_reference_arm_json_line():
-    args = argparse.Namespace(workload="tiny", steps=2, warmup=1)
+    args = argparse.Namespace(workload="tiny", steps=2, warmup=1, ref_seconds=1.0)
     out = bench.run_reference(args, world=1, rank=0)
     for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                 "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
@@ -16,6 +16,9 @@ def test_reference_arm_json_line():
     assert out["metric"] == bench.METRIC and out["steps"] == 2 and out["warmup"] == 1
     cb = out["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == out["value"] and cb["sample"]
+    import os
+
+    assert cb["cores"] == os.cpu_count()  # one oracle process per host core
     e2e = out["e2e"]
     assert e2e["value"] == out["value"] and e2e["unit"] == out["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

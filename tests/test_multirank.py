@@ -32,9 +32,10 @@ def _worker(rank, world, port, q):
 
         bench.barrier(world)
         m = bench.max_over_ranks(10.0 + rank, world)
-        w = bench.rank_workload(WORKLOADS["wan14b"], rank)
         lo, hi = bench.shard_heads(40, world, rank)
-        q.put((rank, m, w.seed, w.philox_seed, lo, hi))
+        weak = bench.rank_heads(WORKLOADS["wan14b"], world, rank, "weak")
+        strong = bench.rank_heads(WORKLOADS["wan14b"], world, rank, "strong")
+        q.put((rank, m, weak, strong, lo, hi))
         bench.barrier(world)
     finally:
         dist.destroy_process_group()
@@ -52,7 +53,9 @@ def test_two_rank_timing_and_sharding():
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(2))
     assert [r[1] for r in res] == [11.0, 11.0]  # max over ranks seen by both
-    assert res[0][2] != res[1][2] and res[0][3] != res[1][3]  # independent layers per rank
+    # weak: a layer of 80 heads, 40 per rank; strong: the 40-head layer split in two
+    assert (res[0][2], res[1][2]) == ((0, 40, 80), (40, 80, 80))
+    assert (res[0][3], res[1][3]) == ((0, 20, 40), (20, 40, 40))
     assert (res[0][4], res[0][5], res[1][4], res[1][5]) == (0, 20, 20, 40)
 
 

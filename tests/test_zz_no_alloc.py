@@ -47,6 +47,10 @@ def test_noalloc_matches_workspace_select_on_two_calls_in_a_row():
     R1 = _with_workspace(p1, Q1, K1, shape1)
     R2 = _with_workspace(p2, Q2, K2, shape2)
     assert ab.ab_get_status() == 0
+    # the same kernels with the same work split: S must match bit for bit (stale scratch
+    # left by call 1 must not leak into call 2)
+    assert torch.equal(S1, R1), "no-alloc call 1 differs from ab_select"
+    assert torch.equal(S2, R2), "no-alloc call 2 differs from ab_select"
     assert_s_close(S1.cpu().numpy(), R1.cpu().double().numpy(), "no-alloc call 1")
     assert_s_close(S2.cpu().numpy(), R2.cpu().double().numpy(), "no-alloc call 2")
 
