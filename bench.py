@@ -376,7 +376,7 @@ def run_ours(args, world, rank, local):
                      "traffic": attn_traffic(w, Hr),
                      "traffic_source_sha256": attn_source_sha256()[:16],
                      "l2_gather_gbs": round(gathered_bytes(w, Hr) / (attn_ms * 1e-3) / 1e9, 1)},
-        "gpu_launches": args.steps * (4 * run_select + run_plan + reuse * run_attn),
+        "gpu_launches": args.steps * (4 * run_select + run_plan + 2 * reuse * run_attn),  # attention: plan check + attention
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -533,7 +533,13 @@ class OraclePool:
         import multiprocessing as mp
 
         self.w = w
-        self.procs = procs or os.cpu_count() or 1
+        if procs is None:  # the cores this process may run on (at most 64 workers)
+            try:
+                procs = len(os.sched_getaffinity(0))
+            except AttributeError:
+                procs = os.cpu_count() or 1
+            procs = max(1, min(64, procs))
+        self.procs = procs
         self.pool = mp.get_context("spawn").Pool(self.procs, _oracle_worker_init, (w.name,))
         # every worker has drawn its inputs and pooled the keys before anything is timed
         pings = self.pool.map(_oracle_worker_ping, range(2 * self.procs), chunksize=1)

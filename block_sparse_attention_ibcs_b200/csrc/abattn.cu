@@ -280,6 +280,14 @@ ab_status run_attn(const Dims& d, const void* Q, const void* K, const void* V, c
   a.trace = trace;
   using L = AttnSmem<D>;
   const unsigned grid = (unsigned)(d.BH * d.nQ);
+  if (!DENSE) {  // plan rows strictly ascending in [0, nK)
+    const long long rows = d.BH * d.nQ;
+    const long long warps_needed = rows;
+    const long long cap = (long long)device_sms() * 8 * (PLAN_CHECK_THREADS / 32);
+    const long long w = warps_needed < cap ? warps_needed : cap;
+    plan_check_kernel<<<(unsigned)((w + PLAN_CHECK_THREADS / 32 - 1) / (PLAN_CHECK_THREADS / 32)),
+                        PLAN_CHECK_THREADS, 0, st>>>(idx, rows, s, (int)d.nK);
+  }
   if (trace) {
     if (cudaFuncSetAttribute(attn_kernel<D, DENSE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              L::ALLOC) != cudaSuccess)

@@ -103,6 +103,35 @@ struct AttnSmem {
 enum { B_QFULL = 0, B_KFULL0 = 1, B_VFULL0 = 4, B_EMPTY0 = 7, B_SFULL = 10, B_SFREE = 11,
        B_PFULL0 = 12, B_PVDONE0 = 14, B_DRAIN = 16 };
 
+// Validation of a plan handed to ab_attn (a separate pass, so the gather warps, which set
+// the attention's pace, carry no extra work): each row must be strictly ascending, which
+// makes every block count once, with entries in [0, nK).  One warp per row (grid-stride);
+// a violation records AB_ERR_DEVICE_CHECK.  The attention itself masks entries outside
+// [0, nK) (they are never gathered); the output of a row that breaks the order is not
+// specified further.
+constexpr int PLAN_CHECK_THREADS = 256;
+
+__global__ void __launch_bounds__(PLAN_CHECK_THREADS) plan_check_kernel(const int32_t* idx, long long rows,
+                                                                         int s, int nK) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (PLAN_CHECK_THREADS / 32);
+  for (long long row = (long long)blockIdx.x * (PLAN_CHECK_THREADS / 32) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const int32_t* r = idx + row * s;
+    int carry = -1;  // last entry of the previous 32 (below every valid entry)
+    bool bad = false;
+    for (int m0 = 0; m0 < s; m0 += 32) {
+      const int m = m0 + lane;
+      const int v = m < s ? __ldg(r + m) : INT_MAX;
+      const int up = __shfl_up_sync(0xffffffffu, v, 1);
+      const int prev = lane == 0 ? carry : up;
+      carry = __shfl_sync(0xffffffffu, v, 31);
+      bad |= m < s && (v < 0 || v >= nK || v <= prev);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) ab_flag(AB_ERR_DEVICE_CHECK);
+  }
+}
+
 template <int D, bool DENSE, bool TRACE>
 __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
   using L = AttnSmem<D>;
@@ -194,31 +223,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         lr[k] = in ? __ldg(a.logpi + plan_off + m) : 0.f;
       }
     };
-    // An entry is used only if it lies in [0, nK) and is above every earlier entry of its
-    // row (plans are strictly ascending, so no block can count twice); any other entry is
-    // masked (-1: its rows become padding) and flags AB_ERR_DEVICE_CHECK.  The earlier
-    // entries' maximum comes from a max-scan over the lanes and the running maximum of the
-    // row's previous tiles (row_max), so the check holds across tile edges.
-    int row_max = INT_MIN;
-    auto check = [&](int t, int (&jr)[4]) {
+    auto check = [&](int (&jr)[4]) {
       bool bad = false;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        if (32 * k >= nb) break;  // warp-uniform: registers past the tile's blocks hold padding
-        const int e = lane + 32 * k;
-        const bool in = e < nb && t * nb + e < a.s;
-        int incl = in ? jr[k] : INT_MIN;  // inclusive max over lanes 0..lane
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl = max(incl, y);
-        }
-        int before = __shfl_up_sync(0xffffffffu, incl, 1);
-        before = max(row_max, lane == 0 ? INT_MIN : before);  // max of the earlier entries
-        const bool ok = jr[k] >= 0 && jr[k] < a.nK && jr[k] > before;
-        bad |= in && !ok;
-        jr[k] = (in && ok) ? jr[k] : (in ? -1 : PAD);
-        row_max = max(row_max, __shfl_sync(0xffffffffu, incl, 31));
+        const bool ok = jr[k] >= 0 && jr[k] < a.nK;
+        bad |= (jr[k] != PAD) && !ok;
+        jr[k] = ok ? jr[k] : -1;
       }
       if (bad) ab_flag(AB_ERR_DEVICE_CHECK);
     };
@@ -239,7 +250,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     };
     if (!DENSE) {
       fetch(0, jc, lc);
-      check(0, jc);
+      check(jc);
     }
 
     int st = 0;  // t % ATTN_STAGES
@@ -318,7 +329,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           jc[k] = jn[k];
           lc[k] = ln[k];
         }
-        check(t + 1, jc);
+        check(jc);
       }
       st = (st + 1 == ATTN_STAGES) ? 0 : st + 1;
       if (p == 0) ev(EV_COPY_ISSUED, t);

@@ -99,6 +99,35 @@ AB_DEV bool fixed_q32(float lam, float sv, uint32_t& q) {
   return x >= 1.0f;
 }
 
+// The same step in a form that runs mostly on the FMA pipe, for lambda < 2^95 (every row
+// but pathological ones).  With L = lambda 2^32 (an exact scaling), y = fl(L S_j) equals
+// fl(lambda S_j) 2^32 exactly while lambda S_j lies in fp32's normal range, and below it
+// both floors are 0.  cvt.rzi.u32 of y is floor(y) = q_j for y < 2^32 (the largest fp32
+// below 2^32 is 2^32 - 256), saturates to 2^32 - 1 for y >= 2^32 (lambda S_j >= 1), and
+// gives 0 for a negative or NaN y.  So over a set of blocks F = sum cvt(y_j) + n_sat, and
+// the saturation test y >= 2^32 is sat(y - (2^32 - 256)), exactly 0 or 1 (NaN: 0).
+constexpr float LAM_FAST_MAX = 39614081257132168796771975168.f;  // 2^95
+constexpr float TWO32F = 4294967296.f;
+constexpr float BELOW_TWO32F = 4294967040.f;
+
+AB_DEV uint32_t f2u_rz(float y) {
+  uint32_t q;
+  asm("cvt.rzi.u32.f32 %0, %1;" : "=r"(q) : "f"(y));
+  return q;
+}
+// 1 if y >= 2^32, else 0 (y an fp32 product as above)
+AB_DEV float sat_flag(float y) {
+  float t;
+  asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(t) : "f"(y), "f"(-BELOW_TWO32F));
+  return t;
+}
+// acc + q as one wide multiply-add
+AB_DEV uint64_t add_wide(uint64_t acc, uint32_t q) {
+  uint64_t r;
+  asm("mad.wide.u32 %0, %1, 1, %2;" : "=l"(r) : "r"(q), "l"(acc));
+  return r;
+}
+
 // Exclusive block scans of two uint64 values in thread order, one pair of barriers;
 // returns this thread's prefixes and the block totals.
 AB_DEV void block_exscan2_u64(uint64_t v0, uint64_t v1, uint64_t* red0, uint64_t* red1,
@@ -251,6 +280,42 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     return v;
   };
 
+  // This thread's part of F(lam): its saturated count and the sum of its other q_j.
+  auto eval_part = [&](float lam, uint32_t& ns, uint64_t& qs) {
+    if (lam < LAM_FAST_MAX) {
+      const float L = __fmul_rn(lam, TWO32F);
+      uint64_t acc = 0;
+      float nsf = 0.f;
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float y = __fmul_rn(L, x4[k]);
+          acc = add_wide(acc, f2u_rz(y));
+          nsf += sat_flag(y);
+        }
+      }
+      ns = (uint32_t)nsf;
+      qs = acc - (uint64_t)ns * 0xFFFFFFFFull;
+    } else {
+      uint32_t n = 0;
+      uint64_t q64 = 0;
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t q;
+          n += fixed_q32(lam, x4[k], q);
+          q64 += q;
+        }
+      }
+      ns = n;
+      qs = q64;
+    }
+  };
+
   // ---- positive blocks and their total score (fewer than s positive blocks = budget
   // unreachable); per-thread sums in compensated fp32, block sum in fp64.  With the row
   // staged in shared memory this pass also copies it there (coalesced, strided).
@@ -362,18 +427,45 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     uint32_t ns[3] = {0u, 0u, 0u};
     uint64_t qs[3] = {0ull, 0ull, 0ull};
     float rest = 0.f;
-    for (int i = c0; i < c1; ++i) {
-      const float4 v = load4(i);
-      const float x4[4] = {v.x, v.y, v.z, v.w};
+    if (l3[2] < LAM_FAST_MAX) {  // block-uniform; see sat_flag above
+      float L3[3], nsf[3] = {0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int c = 0; c < 3; ++c) L3[c] = __fmul_rn(l3[c], TWO32F);
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          uint32_t q;
-          const bool sat = fixed_q32(l3[c], x4[k], q);  // q = 0 when saturated
-          ns[c] += sat;
-          qs[c] += q;
-          if (c == 1 && !sat && x4[k] > 0.f) rest += x4[k];
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int c = 0; c < 3; ++c) {
+            const float y = __fmul_rn(L3[c], x4[k]);
+            const float sat = sat_flag(y);
+            qs[c] = add_wide(qs[c], f2u_rz(y));
+            nsf[c] += sat;
+            // scores unsaturated at b0: x (positive) times 1 - sat; NaN and x <= 0 add 0
+            if (c == 1) rest = fmaf(1.f - sat, fmaxf(x4[k], 0.f), rest);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        ns[c] = (uint32_t)nsf[c];
+        qs[c] -= (uint64_t)ns[c] * 0xFFFFFFFFull;  // the saturated blocks' 2^32 - 1 each
+      }
+    } else {
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int c = 0; c < 3; ++c) {
+            uint32_t q;
+            const bool sat = fixed_q32(l3[c], x4[k], q);  // q = 0 when saturated
+            ns[c] += sat;
+            qs[c] += q;
+            if (c == 1 && !sat && x4[k] > 0.f) rest += x4[k];
+          }
         }
       }
     }
@@ -403,18 +495,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       const uint32_t b2 = __float_as_uint(lf);
       if (lf > 0.f && isfinite(lf) && b2 > lo && b2 < hi) {
         uint64_t f1[1];
-        uint32_t ns2 = 0;
-        uint64_t qs2 = 0;
-        for (int i = c0; i < c1; ++i) {
-          const float4 v = load4(i);
-          const float x4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint32_t q;
-            ns2 += fixed_q32(lf, x4[k], q);
-            qs2 += q;
-          }
-        }
+        uint32_t ns2;
+        uint64_t qs2;
+        eval_part(lf, ns2, qs2);
         f1[0] = ((uint64_t)ns2 << 32) + qs2;
         double none[1] = {0.0};
         block_sums<1, 1>(f1, none, ru, rd, par);
@@ -448,19 +531,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       } else {
         cand = lo + ((hi - lo) >> 1);
       }
-      uint32_t ns2 = 0;
-      uint64_t qs2 = 0;
-      const float lc = __uint_as_float(cand);
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
-        const float x4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t q;
-          ns2 += fixed_q32(lc, x4[k], q);
-          qs2 += q;
-        }
-      }
+      uint32_t ns2;
+      uint64_t qs2;
+      eval_part(__uint_as_float(cand), ns2, qs2);
       uint64_t f1[1] = {((uint64_t)ns2 << 32) + qs2};
       double none[1] = {0.0};
       block_sums<1, 1>(f1, none, ru, rd, par);
@@ -474,22 +547,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         lo_set = true;
       }
     }
-    if (!hi_known) {  // lambda* = +inf (pathological rows): its part of F
-      uint32_t ns2 = 0;
-      uint64_t qs2 = 0;
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
-        const float x4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t q;
-          ns2 += fixed_q32(__uint_as_float(hi), x4[k], q);
-          qs2 += q;
-        }
-      }
-      hi_nsat = ns2;
-      hi_q = qs2;
-    }
+    if (!hi_known) eval_part(__uint_as_float(hi), hi_nsat, hi_q);  // lambda* = +inf (pathological rows)
   }
   const float lam = __uint_as_float(hi);
 
@@ -549,9 +607,34 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     uint64_t o = out_before;
     int32_t* oidx = a.idx + (size_t)row * a.s;
     uint32_t* oraw = reinterpret_cast<uint32_t*>(a.logpi + (size_t)row * a.s);
-    if (reachable && !capped) {
-      // the common case, branch-light: a saturated block has q = 0 here and is drawn; a
-      // block past the row's end (score 0, q = 0) never is
+    if (reachable && !capped && lam < LAM_FAST_MAX) {
+      // the common case, branch-light, with the FMA-pipe form of q (see sat_flag): a
+      // saturated block has q = 0 here and is drawn; a block past the row's end (score 0,
+      // q = 0) never is
+      uint32_t o32 = (uint32_t)out_before;
+      const uint32_t s32 = (uint32_t)a.s;
+      const float L = __fmul_rn(lam, TWO32F);
+      for (int i = c0; i < c1; ++i) {
+        const float4 v = load4(i);
+        const float x4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float y = __fmul_rn(L, x4[k]);
+          const bool sat = y >= TWO32F;
+          const uint32_t q = f2u_rz(sat ? 0.f : y);
+          const bool sel = sat || dist < q;
+          dist -= q;
+          if (sel) {
+            if (o32 < s32) {
+              oidx[o32] = 4 * i + k;
+              oraw[o32] = sat ? 0xFFFFFFFFu : q;  // pi = 1, or q (at most 2^32 - 256)
+            }
+            ++o32;
+          }
+        }
+      }
+    } else if (reachable && !capped) {
+      // the same with the integer form of q (lambda >= 2^95)
       uint32_t o32 = (uint32_t)out_before;
       const uint32_t s32 = (uint32_t)a.s;
       for (int i = c0; i < c1; ++i) {

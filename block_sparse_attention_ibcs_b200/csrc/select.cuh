@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
   __shared__ int cnt[CMAX];
   __shared__ int off[CMAX];
   __shared__ int alive[CMAX];
+  __shared__ int sb[CMAX + 1];  // segment c = rows [sb[c], sb[c+1])
   __shared__ int8_t lab[128];
   __shared__ uint8_t perm[128];
   const int bq = blockIdx.x;  // bh * nQ + i
@@ -131,25 +132,25 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
 
   const uint16_t* qsrc = a.Q + ((size_t)bh * a.N + row0) * D;
   for (int e = tid; e < n * UNITS; e += KM_THREADS) ((uint4*)qs)[e] = __ldg((const uint4*)qsrc + e);
+  if (tid <= CMAX) sb[tid] = (tid <= C) ? tid * n / C : n;  // one division per bound
+  __syncthreads();
   if (tid < CMAX) {
-    const int s0 = tid * n / C, s1 = (tid + 1) * n / C;
-    cnt[tid] = (tid < C) ? s1 - s0 : 0;
-    alive[tid] = (tid < C) && (s1 > s0);
+    cnt[tid] = (tid < C) ? sb[tid + 1] - sb[tid] : 0;
+    alive[tid] = (tid < C) && (sb[tid + 1] > sb[tid]);
   }
   if (tid < 128) {
     int c = -1;
     if (tid < n)
       for (int cc = 0; cc < C; ++cc)
-        if (tid >= cc * n / C && tid < (cc + 1) * n / C) c = cc;
+        if (tid >= sb[cc] && tid < sb[cc + 1]) c = cc;
     lab[tid] = (int8_t)c;
   }
-  __syncthreads();
   // segment means (fp64, exact sums)
   for (int p = tid; p < CMAX * D; p += KM_THREADS) {
     const int c = p / D, dd = p - c * D;
     double acc = 0.0;
     if (c < C) {
-      const int s0 = c * n / C, s1 = (c + 1) * n / C;
+      const int s0 = sb[c], s1 = sb[c + 1];
       for (int r = s0; r < s1; ++r) acc += bf16_to_double(qs[r * D + dd]);
       const int len = s1 - s0;
       if (len > 0) acc = ((len & (len - 1)) == 0) ? acc * (1.0 / (double)len) : acc / (double)len;
@@ -164,15 +165,13 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
     // fp32 copies of the centroids and their squared norms
     for (int p = tid; p < CMAX * D; p += KM_THREADS) cf[p] = (float)c64[p];
     __syncthreads();
-    if (tid < 32) {
+    {  // |c|^2: warp c for centroid c (KM_THREADS / 32 = CMAX warps)
+      const int c = tid >> 5, l = tid & 31;
+      float part = 0.f;
+      for (int dd = l; dd < D; dd += 32) part = fmaf(cf[c * D + dd], cf[c * D + dd], part);
 #pragma unroll
-      for (int c = 0; c < CMAX; ++c) {
-        float part = 0.f;
-        for (int dd = tid; dd < D; dd += 32) part = fmaf(cf[c * D + dd], cf[c * D + dd], part);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (tid == 0) c2[c] = part;
-      }
+      for (int o = 16; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (l == 0) c2[c] = part;
     }
     __syncthreads();
     // assignment (rows >= n take part in the shuffles but are not stored)

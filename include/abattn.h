@@ -175,8 +175,10 @@ ab_status ab_plan_variant(const ab_params* p, const float* S, int s, uint64_t se
  * tokens (tcgen05 MMAs, fp32 accumulation in tensor memory, O rounded to bf16).
  *   idx, logpi  as produced by ab_plan: int32/fp32 [B,H,nQ,s]; each row's idx entries
  *               must lie in [0, nK) and be strictly ascending (so no block counts
- *               twice).  An entry that breaks either rule is masked out (its block gets
- *               weight 0) and the status word records AB_ERR_DEVICE_CHECK.
+ *               twice).  A validation pass before the attention records
+ *               AB_ERR_DEVICE_CHECK in the status word for any row that breaks either
+ *               rule.  Entries outside [0, nK) are never gathered (their block gets
+ *               weight 0); beyond that, O of a flagged row is not specified.
  *   O           bf16 [B,H,N,d] (device, written)                                      */
 ab_status ab_attn(const ab_params* p, const void* Q, const void* K, const void* V,
                   const int32_t* idx, const float* logpi, int s, void* O, void* stream);
