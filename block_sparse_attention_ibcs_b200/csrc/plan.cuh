@@ -251,19 +251,25 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   __shared__ uint64_t ru[2 * 4 * PLAN_WARPS];
   __shared__ double rd[2 * 2 * PLAN_WARPS];
   __shared__ uint64_t row_bar;  // bulk staging of the row
+  __shared__ uint32_t row_U;    // the row's Philox draw
   int par = 0;  // reduction slot set
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
+  if (tid == 0)  // one thread draws; the others read it after the reductions' barriers
+    row_U = philox4x32_10_w0(plan_counter_row(a, row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32), 0u,
+                             (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
   const int nK = a.nK;
   const float* grow = a.S + (size_t)row * nK;
   const bool uniform = a.mode == AB_PLAN_UNIFORM;
   const int nK4 = (nK + 3) >> 2;  // the row in whole float4s (zeros past nK)
   const uint64_t s = (uint64_t)a.s;
   const uint64_t target = s * TWO32;
-  // This thread's contiguous chunk of float4s (an odd count keeps eight consecutive
-  // threads' 16-byte shared loads on distinct banks); every pass after staging walks it.
-  const int per4 = ((nK4 + PLAN_THREADS - 1) / PLAN_THREADS) | 1;
-  const int c0 = min(nK4, tid * per4), c1 = min(nK4, c0 + per4);
+  // This thread's contiguous chunk of float4s, in thread order; every pass after staging
+  // walks it.  The first nK4 % PLAN_THREADS threads take one float4 more, so every thread
+  // has work (an odd count keeps eight consecutive threads' 16-byte shared loads on
+  // distinct banks; the even ones conflict two ways, which costs less than idle lanes).
+  const int base4 = nK4 / PLAN_THREADS, rem4 = nK4 - base4 * PLAN_THREADS;
+  const int c0 = tid * base4 + min(tid, rem4), c1 = c0 + base4 + (tid < rem4 ? 1 : 0);
   auto load4 = [&](int i) -> float4 {
     if (STAGED) return reinterpret_cast<const float4*>(srow_smem)[i];
     float4 v;
@@ -574,8 +580,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   uint64_t sat_before, rest_before, n_sat, tot_rest;
   block_exscan2_1b(my_sat, my_rest, ru, par, sat_before, rest_before, n_sat, tot_rest);
 
-  const uint32_t U = philox4x32_10_w0(plan_counter_row(a, row), (uint32_t)a.offset, (uint32_t)(a.offset >> 32),
-                                      0u, (uint32_t)a.seed, (uint32_t)(a.seed >> 32));
+  const uint32_t U = row_U;  // written before the first barrier
   // lattice points U + k 2^32 below x, for 0 <= x <= s 2^32 (U < 2^32)
   const uint64_t CB = TWO32 - 1u - (uint64_t)U;
   auto below = [&](uint64_t x) -> uint64_t { return (x + CB) >> 32; };
