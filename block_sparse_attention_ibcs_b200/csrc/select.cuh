@@ -145,17 +145,45 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
         if (tid >= sb[cc] && tid < sb[cc + 1]) c = cc;
     lab[tid] = (int8_t)c;
   }
-  // segment means (fp64, exact sums)
-  for (int p = tid; p < CMAX * D; p += KM_THREADS) {
-    const int c = p / D, dd = p - c * D;
-    double acc = 0.0;
-    if (c < C) {
-      const int s0 = sb[c], s1 = sb[c + 1];
-      for (int r = s0; r < s1; ++r) acc += bf16_to_double(qs[r * D + dd]);
+  // segment means (fp64, exact sums, so the order of the additions does not matter):
+  // thread (segment, dimension pair) loads both dimensions of a row at once and keeps four
+  // partial sums per dimension, so the loads and adds of four rows are in flight together
+  {
+    const uint32_t* qs32 = (const uint32_t*)qs;
+    for (int p2 = tid; p2 < CMAX * (D / 2); p2 += KM_THREADS) {
+      const int c = p2 / (D / 2), dp = p2 - c * (D / 2);
+      double ea[4] = {0.0, 0.0, 0.0, 0.0}, eb[4] = {0.0, 0.0, 0.0, 0.0};  // dimensions 2dp, 2dp + 1
+      const int s0 = c < C ? sb[c] : 0, s1 = c < C ? sb[c + 1] : 0;
+      int r = s0;
+      for (; r + 3 < s1; r += 4) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) wv[k] = qs32[(r + k) * (D / 2) + dp];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          ea[k] += (double)__uint_as_float(wv[k] << 16);
+          eb[k] += (double)__uint_as_float(wv[k] & 0xffff0000u);
+        }
+      }
+      for (; r < s1; ++r) {  // the ragged tail (exact sums: any partial will do)
+        const uint32_t w = qs32[r * (D / 2) + dp];
+        ea[0] += (double)__uint_as_float(w << 16);
+        eb[0] += (double)__uint_as_float(w & 0xffff0000u);
+      }
+      double sa = (ea[0] + ea[1]) + (ea[2] + ea[3]), sbb = (eb[0] + eb[1]) + (eb[2] + eb[3]);
       const int len = s1 - s0;
-      if (len > 0) acc = ((len & (len - 1)) == 0) ? acc * (1.0 / (double)len) : acc / (double)len;
+      if (len > 0) {
+        if ((len & (len - 1)) == 0) {
+          sa *= 1.0 / (double)len;
+          sbb *= 1.0 / (double)len;
+        } else {
+          sa /= (double)len;
+          sbb /= (double)len;
+        }
+      }
+      c64[c * D + 2 * dp] = sa;
+      c64[c * D + 2 * dp + 1] = sbb;
     }
-    c64[p] = acc;
   }
   __syncthreads();
 
@@ -274,14 +302,27 @@ __global__ void __launch_bounds__(KM_THREADS) kmeans_kernel(SelectArgs a) {
       for (int c = 0; c < CMAX; ++c) {
         const int k = cnt[c];  // block-uniform
         if (k > 0) {
-          double acc = 0.0;
-          for (int q = r0 + h; q < r0 + k; q += PARTS) acc += bf16_to_double(qs[perm[q] * D + dd]);
+          double acc0 = 0.0, acc1 = 0.0;  // two partial sums: two members' loads in flight
+          int q = r0 + h;
+          for (; q + PARTS < r0 + k; q += 2 * PARTS) {
+            const int ra = perm[q], rb = perm[q + PARTS];
+            acc0 += bf16_to_double(qs[ra * D + dd]);
+            acc1 += bf16_to_double(qs[rb * D + dd]);
+          }
+          if (q < r0 + k) acc0 += bf16_to_double(qs[perm[q] * D + dd]);
+          double acc = acc0 + acc1;
 #pragma unroll
           for (int o = 1; o < PARTS; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          if (h == 0) c64[c * D + dd] = acc / (double)k;
+          if (h == 0) c64[c * D + dd] = acc;  // the member sum; divided below
         }
         r0 += k;
       }
+    }
+    __syncthreads();
+    // member means: the 1024 divisions spread over all threads (independent of each other)
+    for (int p = tid; p < CMAX * D; p += KM_THREADS) {
+      const int k = cnt[p / D];
+      if (k > 0) c64[p] = c64[p] / (double)k;
     }
     __syncthreads();
     if (tid < CMAX) alive[tid] = cnt[tid] > 0;
