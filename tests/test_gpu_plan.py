@@ -164,3 +164,28 @@ def test_plan_stress_rows_every_path():
     for s in (1, 7, 64, 200):
         idx, lp = _gpu_plan(p, St, s, 77, 5)
         _check_rows(S, idx, lp, s, 77, 5, range(R))
+
+
+@pytest.mark.parametrize("nK", [28_672, 28_676, 28_677])
+def test_plan_rows_at_the_staging_limit(nK):
+    """Rows of exactly the planner's staging limit (staged in shared memory) and just past
+    it (re-read from global memory on every pass), with nK a multiple of 4 and odd: both
+    paths draw the oracle's plan.  A stress mix of rows: heavy tails, a saturated block,
+    zeros, NaN."""
+    rng = np.random.default_rng(nK)
+    N = 4 * nK  # KV blocks of 4 tokens
+    nQ = -(-N // 128)
+    R = 6  # rows checked; the launch covers all nQ rows of one head
+    S = torch.from_numpy(np.abs(rng.standard_normal((nQ, nK))).astype(np.float32) ** 3)
+    rows = []
+    x = np.exp(3 * rng.standard_normal(nK)); rows.append(x / x.sum())
+    y = np.full(nK, 1e-6); y[nK - 2] = 0.5; rows.append(y / y.sum())      # saturated in the tail
+    z = rng.random(nK); z[: nK // 2] = 0.0; rows.append(z)                  # zeros up front
+    t = rng.random(nK) ** 9; t[nK - 1] = np.nan; rows.append(t)             # NaN at the end
+    u = np.full(nK, 1.0); rows.append(u)                                    # flat
+    v = rng.dirichlet(np.full(nK, 0.2)); rows.append(v)
+    S[:R] = torch.from_numpy(np.stack(rows).astype(np.float32))
+    p = ab.params(1, 1, N, 64, kv_block=4)
+    for s in (64, 2048):
+        idx, lp = _gpu_plan(p, S.cuda().reshape(1, 1, nQ, nK), s, 31, 2)
+        _check_rows(S.numpy(), idx, lp, s, 31, 2, list(range(R)) + [nQ - 1])
