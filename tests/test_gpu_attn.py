@@ -184,6 +184,28 @@ def test_non_ascending_plan_rows_are_flagged():
     assert ab.ab_get_status() == 0
 
 
+@pytest.mark.parametrize("s,m", [(256, 128), (256, 255), (33, 17), (33, 32)])
+def test_plan_validation_across_steps_and_odd_budgets(s, m):
+    """The validation pass reads four entries per lane (a 128-entry step per warp) when the
+    rows are 16-byte aligned, one per lane otherwise: a repeated entry is found at a step
+    boundary, at the row's end, and with an odd budget s."""
+    H, N, d, bk = 1, 1024, 64, 4
+    Q, K, V = _qkv(H, N, d, seed=19)
+    nQ, nK = N // 128, N // bk
+    rng = np.random.default_rng(s + m)
+    good = torch.from_numpy(np.stack([np.sort(rng.choice(nK, s, replace=False))
+                                      for _ in range(nQ)]).astype(np.int32))
+    lp = torch.zeros(nQ, s)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    O_ = torch.empty(Q.shape, dtype=torch.bfloat16, device="cuda")
+    ab.ab_attn(p, Q.cuda(), K.cuda(), V.cuda(), good.cuda(), lp.cuda(), s, O_)
+    assert ab.ab_get_status() == 0
+    bad = good.clone()
+    bad[5, m] = bad[5, m - 1]
+    ab.ab_attn(p, Q.cuda(), K.cuda(), V.cuda(), bad.cuda(), lp.cuda(), s, O_)
+    assert ab.ab_get_status() == -7
+
+
 def test_device_wait_timeout_is_reported_and_context_survives():
     """A producer that never signals tile 0: the bounded waits give up after 50 ms, the
     status word reports AB_ERR_DEVICE_TIMEOUT, and the context stays usable."""
