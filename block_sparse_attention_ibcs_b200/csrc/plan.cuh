@@ -189,19 +189,18 @@ AB_DEV void block_sums(uint64_t (&u)[NU], double (&dv)[ND], uint64_t* ru, double
     for (int k = 0; k < ND; ++k) sd[k * PLAN_WARPS + w] = dv[k];
   }
   __syncthreads();
+  // the 16 warp partials: lane l (and l + 16) takes warp l's, then a 16-lane shuffle tree
+  static_assert(PLAN_WARPS == 16, "one warp partial per half-warp lane");
 #pragma unroll
-  for (int k = 0; k < NU; ++k) {
-    uint64_t t = 0;
+  for (int k = 0; k < NU; ++k) u[k] = su[k * PLAN_WARPS + (l & 15)];
 #pragma unroll
-    for (int i = 0; i < PLAN_WARPS; ++i) t += su[k * PLAN_WARPS + i];
-    u[k] = t;
-  }
+  for (int k = 0; k < ND; ++k) dv[k] = sd[k * PLAN_WARPS + (l & 15)];
 #pragma unroll
-  for (int k = 0; k < ND; ++k) {
-    double t = 0.0;
+  for (int o = 8; o; o >>= 1) {
 #pragma unroll
-    for (int i = 0; i < PLAN_WARPS; ++i) t += sd[k * PLAN_WARPS + i];
-    dv[k] = t;
+    for (int k = 0; k < NU; ++k) u[k] += __shfl_xor_sync(0xffffffffu, u[k], o);
+#pragma unroll
+    for (int k = 0; k < ND; ++k) dv[k] += __shfl_xor_sync(0xffffffffu, dv[k], o);
   }
   par ^= 1;
 }
@@ -227,21 +226,24 @@ AB_DEV void block_exscan2_1b(uint64_t v0, uint64_t v1, uint64_t* ru, int& par, u
     su[PLAN_WARPS + w] = inc1;
   }
   __syncthreads();
-  uint64_t b0 = 0, b1 = 0, t0 = 0, t1 = 0;
+  // the 16 warp totals: lane l (and l + 16) takes warp l's, an inclusive 16-lane scan, then
+  // the scan at lane w - 1 is what the warps before this one hold, at lane 15 the total
+  uint64_t x0 = su[l & 15], x1 = su[PLAN_WARPS + (l & 15)];
 #pragma unroll
-  for (int i = 0; i < PLAN_WARPS; ++i) {
-    const uint64_t x0 = su[i], x1 = su[PLAN_WARPS + i];
-    if (i < w) {
-      b0 += x0;
-      b1 += x1;
+  for (int o = 1; o < 16; o <<= 1) {
+    const uint64_t y0 = __shfl_up_sync(0xffffffffu, x0, o, 16);
+    const uint64_t y1 = __shfl_up_sync(0xffffffffu, x1, o, 16);
+    if ((l & 15) >= o) {
+      x0 += y0;
+      x1 += y1;
     }
-    t0 += x0;
-    t1 += x1;
   }
-  before0 = b0 + inc0 - v0;
-  before1 = b1 + inc1 - v1;
-  total0 = t0;
-  total1 = t1;
+  const uint64_t p0 = __shfl_sync(0xffffffffu, x0, w > 0 ? w - 1 : 0);
+  const uint64_t p1 = __shfl_sync(0xffffffffu, x1, w > 0 ? w - 1 : 0);
+  total0 = __shfl_sync(0xffffffffu, x0, 15);
+  total1 = __shfl_sync(0xffffffffu, x1, 15);
+  before0 = (w > 0 ? p0 : 0ull) + inc0 - v0;
+  before1 = (w > 0 ? p1 : 0ull) + inc1 - v1;
   par ^= 1;
 }
 
