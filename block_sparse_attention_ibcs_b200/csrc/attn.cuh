@@ -75,7 +75,7 @@ struct AttnArgs {
 // Event tracing (TRACE builds only): CTAs 0, 1 and the one at a third of the grid record
 // clock64() per tile for the events below into trace[((slot * 16) + event) * 128 + t].
 enum { EV_COPY_START = 0, EV_COPY_ISSUED, EV_SM_LOADED, EV_SM_MAX, EV_LANDED, EV_QK,
-       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_UNUSED12,
+       EV_SM_PBUF, EV_PV, EV_SM_START, EV_SM_READY, EV_SM_PDONE, EV_END, EV_V_LANDED,
        EV_SM_PDONE_W1, EV_SM_PDONE_W2, EV_SM_PDONE_W3, EV_COUNT };
 constexpr int TRACE_TILES = 128;
 
@@ -364,9 +364,17 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
       tc_fence_after();
       int nqk = 0, npv = 0;              // next QK / PV to issue (npv < nqk)
       int sq = 0, sp = 0;                // their ring stages (t % 3)
+      int nv = 0;                        // TRACE: next tile whose V arrival is to be seen
       uint64_t t_last = globaltimer_ns();
       while (ok && npv < T) {
         bool progressed = false;
+        // TRACE: V(nv) is polled once its K has landed and before PV(nv) is issued, so the
+        // stage's barrier cannot be a phase ahead (V(nv + 3) waits for PV(nv))
+        if (TRACE && nv < nqk && nv >= npv && nv < T &&
+            mbar_test(&bars[B_VFULL0 + nv % ATTN_STAGES], (nv / ATTN_STAGES) & 1)) {
+          ev(EV_V_LANDED, nv);
+          ++nv;
+        }
         if (npv < nqk && mbar_test(&bars[B_PFULL0 + (npv & 1)], (npv >> 1) & 1) &&
             mbar_test(&bars[B_VFULL0 + sp], (npv / ATTN_STAGES) & 1)) {
           fence_proxy_async_smem();
@@ -379,6 +387,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
           umma_commit(&bars[B_PVDONE0 + (npv & 1)]);
           umma_commit(&bars[B_EMPTY0 + sp]);
           ev(EV_PV, npv);
+          if (TRACE && nv == npv) {  // seen here first
+            ev(EV_V_LANDED, nv);
+            ++nv;
+          }
           ++npv;
           sp = (sp + 1 == ATTN_STAGES) ? 0 : sp + 1;
           progressed = true;

@@ -196,14 +196,14 @@ ab_status ab_attn_dense(const ab_params* p, const void* Q, const void* K, const 
  *  - trace (device, may be NULL; 8-byte aligned, 3*16*128 uint64, zeroed by the caller):
  *    a separately compiled traced kernel records clock64() for each pipeline event of
  *    tiles 0..127 of CTAs 0, 1 and gridDim/3, at trace[(slot*16 + event)*128 + tile];
- *    events (producer warps: 0, 1; MMA warp: 4, 5, 7; softmax warps: the rest):
+ *    events (producer warps: 0, 1; MMA warp: 4, 5, 7, 12; softmax warps: the rest):
  *      0 the tile's copies start (its ring stage is free)   1 all its copies are issued
  *      2 S loaded from tensor memory                         3 exponentials done (P built)
  *      4 K rows and shifts landed (seen by the MMA warp)     5 QK MMAs issued
  *      6 the P buffer is free (PV two tiles back done)       7 PV MMAs issued
  *      8 softmax tile start                                  9 S ready (QK done)
  *      10 P stored by warp 0                                 11 CTA end (tile slot 0)
- *      12 unused                                             13, 14, 15 P stored by warps 1, 2, 3
+ *      12 V rows landed (seen by the MMA warp)               13, 14, 15 P stored by warps 1, 2, 3
  * With skip_first_arrival = 0 and trace = NULL it is ab_attn with another wait limit.   */
 ab_status ab_attn_debug(const ab_params* p, const void* Q, const void* K, const void* V,
                         const int32_t* idx, const float* logpi, int s, void* O,

@@ -221,3 +221,33 @@ def test_device_wait_timeout_is_reported_and_context_survives():
     ab.ab_attn_debug(*args, 0, 2_000_000_000)
     assert ab.ab_get_status() == 0
     _check(O_.cpu(), Q, K, V, idx, lp, H, N, bk)
+
+
+def test_traced_kernel_matches_and_orders_its_events():
+    """The traced kernel (ab_attn_debug with a trace buffer) gives the untraced O bit for bit,
+    and each traced tile's events come in pipeline order: copies start before they are all
+    issued; K and V land after the copies are issued; QK is issued after K landed; PV after
+    V landed and after every softmax warp stored P."""
+    H, N, d, bk, s = 2, 8192, 128, 4, 512  # 64 query blocks, 16 tiles each
+    Q, K, V = _qkv(H, N, d, seed=21)
+    nQ = N // 128
+    idx, lp = random_plan(H * nQ, N // bk, s, seed=4)
+    p = ab.params(1, H, N, d, kv_block=bk)
+    O_ref = _run(p, Q, K, V, idx, lp, s)
+    O_tr = torch.empty_like(O_ref)
+    tr = torch.zeros(3 * 16 * 128, dtype=torch.int64, device="cuda")
+    ab.ab_attn_debug(p, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), lp.cuda(), s, O_tr, 0, 2_000_000_000, tr)
+    assert ab.ab_get_status() == 0
+    assert torch.equal(O_tr, O_ref)
+    ev = tr.view(3, 16, 128).cpu().numpy()
+    T = s * bk // 128
+    for slot in range(3):
+        e = ev[slot][:, :T]
+        assert (e[[0, 1, 2, 3, 4, 5, 7, 8, 9, 10, 12, 13, 14, 15]] > 0).all(), f"slot {slot}: missing events"
+        assert (e[1] >= e[0]).all()
+        assert (e[4] >= e[1]).all() and (e[12] >= e[1]).all()
+        assert (e[5] >= e[4]).all()
+        assert (e[7] >= e[12]).all()
+        for w in (10, 13, 14, 15):
+            assert (e[7] >= e[w]).all(), f"slot {slot}: PV before P of warp event {w}"
+        assert (e[9] >= e[5]).all() and (e[2] >= e[9]).all() and (e[3] >= e[2]).all()
