@@ -187,8 +187,8 @@ def attn_source_sha256():
 # (dram__bytes_read.sum + dram__bytes_write.sum of the Wan2.1-1.3B-shaped launch, scaled by
 # the number of heads: every head's K, V, Q and O cross DRAM once), valid only for the
 # kernel source it was taken on; `roofline.traffic` is null for any other source.
-ATTN_TRAFFIC = {"bytes_wan14b": 1.0415e9 * 40 / 12, "captured_heads": 12,
-                "source_sha256": "74f343e22ad043df6ea7d9759c52ae835486d547238eba3b50f23a518581b135"}
+ATTN_TRAFFIC = {"bytes_wan14b": 1.0385e9 * 40 / 12, "captured_heads": 12,
+                "source_sha256": "9859efbd2b44054afd8d36c13896fbc5c2c29d6fb2033817e91b61716d6adebf"}
 
 
 def attn_traffic(w, heads):
