@@ -245,8 +245,12 @@ ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t
   if (d.nK <= PLAN_STAGE_MAX_FLOATS) {
     const size_t smem = (size_t)((d.nK + 3) / 4) * 16;  // row padded to whole float4s
     // per-device attribute; cheap enough to set on every launch
+    // and the largest shared-memory carveout: a Wan-sized row (75.6 KB) then fits three
+    // rows per SM
     if (cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PLAN_SMEM_MAX_FLOATS * 4) != cudaSuccess)
+                             PLAN_SMEM_MAX_FLOATS * 4) != cudaSuccess ||
+        cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return launch_status();
     plan_kernel<true><<<rows, PLAN_THREADS, smem, st>>>(a);
   } else {

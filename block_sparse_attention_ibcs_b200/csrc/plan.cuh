@@ -170,8 +170,13 @@ AB_DEV void block_exscan2_u64(uint64_t v0, uint64_t v1, uint64_t* red0, uint64_t
 // writes its partials into the slot set `par`, which alternates between calls, so a call
 // never overwrites slots that a thread may still be reading from the call before (every
 // thread has left that call's reads before it reaches this call's barrier).
+// Slots per set: at most PLAN_RED_U uint64 and PLAN_RED_D double values per reduction (kept
+// small: with a staged Wan-sized row, three rows per SM fit in shared memory only so).
+constexpr int PLAN_RED_U = 3, PLAN_RED_D = 1;
+
 template <int NU, int ND>
 AB_DEV void block_sums(uint64_t (&u)[NU], double (&dv)[ND], uint64_t* ru, double* rd, int& par) {
+  static_assert(NU <= PLAN_RED_U && ND <= PLAN_RED_D, "reduction slots");
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -180,8 +185,8 @@ AB_DEV void block_sums(uint64_t (&u)[NU], double (&dv)[ND], uint64_t* ru, double
 #pragma unroll
     for (int k = 0; k < ND; ++k) dv[k] += __shfl_xor_sync(0xffffffffu, dv[k], o);
   }
-  uint64_t* su = ru + par * 4 * PLAN_WARPS;
-  double* sd = rd + par * 2 * PLAN_WARPS;
+  uint64_t* su = ru + par * PLAN_RED_U * PLAN_WARPS;
+  double* sd = rd + par * PLAN_RED_D * PLAN_WARPS;
   if (l == 0) {
 #pragma unroll
     for (int k = 0; k < NU; ++k) su[k * PLAN_WARPS + w] = u[k];
@@ -220,7 +225,8 @@ AB_DEV void block_exscan2_1b(uint64_t v0, uint64_t v1, uint64_t* ru, int& par, u
       inc1 += y1;
     }
   }
-  uint64_t* su = ru + par * 4 * PLAN_WARPS;
+  static_assert(PLAN_RED_U >= 2, "two scans per set");
+  uint64_t* su = ru + par * PLAN_RED_U * PLAN_WARPS;
   if (l == 31) {
     su[w] = inc0;
     su[PLAN_WARPS + w] = inc1;
@@ -250,8 +256,8 @@ AB_DEV void block_exscan2_1b(uint64_t v0, uint64_t v1, uint64_t* ru, int& par, u
 template <bool STAGED>
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   extern __shared__ float srow_smem[];
-  __shared__ uint64_t ru[2 * 4 * PLAN_WARPS];
-  __shared__ double rd[2 * 2 * PLAN_WARPS];
+  __shared__ uint64_t ru[2 * PLAN_RED_U * PLAN_WARPS];
+  __shared__ double rd[2 * PLAN_RED_D * PLAN_WARPS];
   __shared__ uint64_t row_bar;  // bulk staging of the row
   __shared__ uint32_t row_U;    // the row's Philox draw
   int par = 0;  // reduction slot set
