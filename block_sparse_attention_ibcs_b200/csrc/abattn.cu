@@ -242,19 +242,19 @@ ab_status run_plan(const Dims& d, const float* S, int s, uint64_t seed, uint64_t
     }
     return launch_status();
   }
-  if (d.nK <= PLAN_STAGE_MAX_FLOATS) {
-    const size_t smem = (size_t)((d.nK + 3) / 4) * 16;  // row padded to whole float4s
-    // per-device attribute; cheap enough to set on every launch
-    // and the largest shared-memory carveout: a Wan-sized row (75.6 KB) then fits three
-    // rows per SM
-    if (cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PLAN_SMEM_MAX_FLOATS * 4) != cudaSuccess ||
-        cudaFuncSetAttribute(plan_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+  {
+    const int nK4 = (int)((d.nK + 3) / 4);
+    const size_t smem = (size_t)(nK4 < PLAN_STAGE_FLOAT4S ? nK4 : PLAN_STAGE_FLOAT4S) * 16;  // staged part
+    // per-device attributes, cheap enough to set on every launch; the largest
+    // shared-memory carveout fits three staged rows per SM
+    const bool whole = nK4 <= PLAN_STAGE_FLOAT4S;
+    auto kern = whole ? plan_kernel<1> : plan_kernel<2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PLAN_STAGE_FLOAT4S * 16) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return launch_status();
-    plan_kernel<true><<<rows, PLAN_THREADS, smem, st>>>(a);
-  } else {
-    plan_kernel<false><<<rows, PLAN_THREADS, 0, st>>>(a);
+    kern<<<rows, PLAN_THREADS, smem, st>>>(a);
   }
   return launch_status();
 }

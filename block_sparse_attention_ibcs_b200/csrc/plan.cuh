@@ -35,11 +35,12 @@ namespace abattn {
 constexpr int PLAN_THREADS = 512;
 constexpr int PLAN_WARPS = PLAN_THREADS / 32;
 constexpr int PLAN_SMEM_MAX_FLOATS = 40 * 1024;  // 160 KB of staged row (top-k keys)
-// The SIP planner stages a row only while two CTAs still fit on an SM (112 KB each):
-// measured on B200, one staged CTA per SM (e.g. 29,700 blocks) is slower than re-reading
-// the row from L2 with two CTAs per SM (4.9 vs 4.0 ms at the HunyuanVideo shape), while at
-// 18,900 blocks staging wins (2.7 vs 3.6 ms).
-constexpr int PLAN_STAGE_MAX_FLOATS = 28 * 1024;
+// The SIP planner stages at most the first PLAN_STAGE_FLOAT4S float4s of a row (75,760
+// bytes) in shared memory, so that three rows fit on an SM (228 KB, less the 1,040 bytes of
+// static shared memory and the 1 KB the system reserves per block); a longer row reads its
+// tail from global memory.  Measured on B200: three rows per SM instead of two took the
+// Wan2.1-14B planner (18,900 blocks, fully staged) from 1.90 to 1.64 ms.
+constexpr int PLAN_STAGE_FLOAT4S = 4735;
 constexpr uint64_t TWO32 = 1ull << 32;
 constexpr uint64_t kPlanTimeoutNs = 2000000000ull;  // bounded wait for the staged row
 
@@ -253,8 +254,10 @@ AB_DEV void block_exscan2_1b(uint64_t v0, uint64_t v1, uint64_t* ru, int& par, u
   par ^= 1;
 }
 
-template <bool STAGED>
-__global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
+// MODE 1: the whole row is staged in shared memory; MODE 2: its first PLAN_STAGE_FLOAT4S
+// float4s are, and the rest is read from global memory on every pass.
+template <int MODE>
+__global__ void __launch_bounds__(PLAN_THREADS, 3) plan_kernel(PlanArgs a) {
   extern __shared__ float srow_smem[];
   __shared__ uint64_t ru[2 * PLAN_RED_U * PLAN_WARPS];
   __shared__ double rd[2 * PLAN_RED_D * PLAN_WARPS];
@@ -278,8 +281,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   // distinct banks; the even ones conflict two ways, which costs less than idle lanes).
   const int base4 = nK4 / PLAN_THREADS, rem4 = nK4 - base4 * PLAN_THREADS;
   const int c0 = tid * base4 + min(tid, rem4), c1 = c0 + base4 + (tid < rem4 ? 1 : 0);
-  auto load4 = [&](int i) -> float4 {
-    if (STAGED) return reinterpret_cast<const float4*>(srow_smem)[i];
+  // The row's first ns4 float4s are staged in shared memory (all of it in MODE 1); the rest
+  // is read from global memory, 16 bytes at a time when the row is 16-byte aligned and a
+  // whole number of float4s.
+  const int ns4 = MODE == 1 ? nK4 : min(nK4, PLAN_STAGE_FLOAT4S);
+  const bool gvec = !uniform && ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
+  auto gload4 = [&](int i) -> float4 {
+    if (gvec) return __ldg(reinterpret_cast<const float4*>(grow) + i);
     float4 v;
     const int j = 4 * i;
     if (uniform) {
@@ -293,6 +301,16 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
     }
     return v;
   };
+  // Every pass walks this thread's chunk: its staged part from shared memory, then the rest.
+  const int cm = min(max(ns4, c0), c1);
+  auto walk = [&](auto&& body) {
+    if (MODE == 1) {
+      for (int i = c0; i < c1; ++i) body(i, reinterpret_cast<const float4*>(srow_smem)[i]);
+    } else {
+      for (int i = c0; i < cm; ++i) body(i, reinterpret_cast<const float4*>(srow_smem)[i]);
+      for (int i = cm; i < c1; ++i) body(i, gload4(i));
+    }
+  };
 
   // This thread's part of F(lam): its saturated count and the sum of its other q_j.
   auto eval_part = [&](float lam, uint32_t& ns, uint64_t& qs) {
@@ -300,8 +318,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       const float L = __fmul_rn(lam, TWO32F);
       uint64_t acc = 0;
       float nsf = 0.f;
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -309,14 +326,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
           acc = add_wide(acc, f2u_rz(y));
           nsf += sat_flag(y);
         }
-      }
+      });
       ns = (uint32_t)nsf;
       qs = acc - (uint64_t)ns * 0xFFFFFFFFull;
     } else {
       uint32_t n = 0;
       uint64_t q64 = 0;
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -324,7 +340,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
           n += fixed_q32(lam, x4[k], q);
           q64 += q;
         }
-      }
+      });
       ns = n;
       qs = q64;
     }
@@ -345,18 +361,18 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         ++npos;
       }
     };
-    const bool bulk = STAGED && !uniform && ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
+    const bool bulk = !uniform && ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
     if (bulk) {
       // the whole row in one bulk copy (one request in flight instead of a dependent
       // chain of loads per thread), then the sums over this thread's chunk
       if (tid == 0) {
         mbar_init(&row_bar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&row_bar, (uint32_t)nK * 4u);
+        mbar_arrive_expect_tx(&row_bar, (uint32_t)ns4 * 16u);
         asm volatile(
             "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                 smem_u32(srow_smem)),
-            "l"(grow), "r"((uint32_t)nK * 4u), "r"(smem_u32(&row_bar))
+            "l"(grow), "r"((uint32_t)ns4 * 16u), "r"(smem_u32(&row_bar))
             : "memory");
       }
       __syncthreads();  // the barrier is initialised before anyone waits on it
@@ -365,14 +381,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
         if (tid == 0) ab_flag(AB_ERR_DEVICE_TIMEOUT);
         return;
       }
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = reinterpret_cast<const float4*>(srow_smem)[i];
+      walk([&](const int i, const float4 v) {
         acc(v.x);
         acc(v.y);
         acc(v.z);
         acc(v.w);
-      }
-    } else if (STAGED) {
+      });
+    } else {
       const bool vec = ((uintptr_t)grow & 15u) == 0 && (nK & 3) == 0;
       float4* s4 = reinterpret_cast<float4*>(srow_smem);
       for (int j = tid; j < nK4; j += PLAN_THREADS) {
@@ -390,21 +405,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
           v.z = (4 * j + 2 < nK) ? __ldg(grow + 4 * j + 2) : 0.f;
           v.w = (4 * j + 3 < nK) ? __ldg(grow + 4 * j + 3) : 0.f;
         }
-        s4[j] = v;
+        if (j < ns4) s4[j] = v;
         acc(v.x);
         acc(v.y);
         acc(v.z);
         acc(v.w);
       }
       // read by other threads only after the barrier of the block sum below
-    } else {
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
-        acc(v.x);
-        acc(v.y);
-        acc(v.z);
-        acc(v.w);
-      }
     }
     tot = (double)sum - (double)comp;
   }
@@ -445,8 +452,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       float L3[3], nsf[3] = {0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 3; ++c) L3[c] = __fmul_rn(l3[c], TWO32F);
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -460,15 +466,14 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
             if (c == 1) rest = fmaf(1.f - sat, fmaxf(x4[k], 0.f), rest);
           }
         }
-      }
+      });
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
         ns[c] = (uint32_t)nsf[c];
         qs[c] -= (uint64_t)ns[c] * 0xFFFFFFFFull;  // the saturated blocks' 2^32 - 1 each
       }
     } else {
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
             if (c == 1 && !sat && x4[k] > 0.f) rest += x4[k];
           }
         }
-      }
+      });
     }
     uint64_t f3[3];
 #pragma unroll
@@ -575,15 +580,14 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
   } else {
     my_sat = 0;
     my_rest = 0;
-    for (int i = c0; i < c1; ++i) {
-      const float4 v = load4(i);
+    walk([&](const int i, const float4 v) {
       const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (4 * i + k >= nK) break;
         if (x4[k] > 0.f) ++my_sat; else ++my_rest;
       }
-    }
+    });
   }
   uint64_t sat_before, rest_before, n_sat, tot_rest;
   block_exscan2_1b(my_sat, my_rest, ru, par, sat_before, rest_before, n_sat, tot_rest);
@@ -627,8 +631,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
       uint32_t o32 = (uint32_t)out_before;
       const uint32_t s32 = (uint32_t)a.s;
       const float L = __fmul_rn(lam, TWO32F);
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -645,13 +648,12 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
             ++o32;
           }
         }
-      }
+      });
     } else if (reachable && !capped) {
       // the same with the integer form of q (lambda >= 2^95)
       uint32_t o32 = (uint32_t)out_before;
       const uint32_t s32 = (uint32_t)a.s;
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -667,10 +669,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
             ++o32;
           }
         }
-      }
+      });
     } else {
-      for (int i = c0; i < c1; ++i) {
-        const float4 v = load4(i);
+      walk([&](const int i, const float4 v) {
         const float x4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -703,7 +704,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(PlanArgs a) {
             ++o;
           }
         }
-      }
+      });
     }
   }
   // log(pi) for the s outputs, spread evenly over the threads (no divergent fp64 log)

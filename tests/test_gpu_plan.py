@@ -166,12 +166,13 @@ def test_plan_stress_rows_every_path():
         _check_rows(S, idx, lp, s, 77, 5, range(R))
 
 
-@pytest.mark.parametrize("nK", [28_672, 28_676, 28_677])
+@pytest.mark.parametrize("nK", [18_940, 18_941, 18_944, 28_677, 29_700])
 def test_plan_rows_at_the_staging_limit(nK):
-    """Rows of exactly the planner's staging limit (staged in shared memory) and just past
-    it (re-read from global memory on every pass), with nK a multiple of 4 and odd: both
-    paths draw the oracle's plan.  A stress mix of rows: heavy tails, a saturated block,
-    zeros, NaN."""
+    """Rows of exactly the planner's staging size (18,940 scores, the whole row in shared
+    memory) and past it (the first 18,940 staged, the tail re-read from global memory on
+    every pass), with nK a multiple of 4 (one bulk copy; 16-byte tail loads) and odd
+    (strided staging; scalar tail loads), up to a HunyuanVideo-length row: every path draws
+    the oracle's plan.  A stress mix of rows: heavy tails, a saturated block, zeros, NaN."""
     rng = np.random.default_rng(nK)
     N = 4 * nK  # KV blocks of 4 tokens
     nQ = -(-N // 128)
