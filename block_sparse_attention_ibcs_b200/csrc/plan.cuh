@@ -15,8 +15,9 @@
 //   its interval, with U = word 0 of Philox4x32-10(key = seed, counter = (row, offset_lo,
 //   offset_hi, 0)).
 //
-// One CTA of PLAN_THREADS threads per row.  The row is staged in shared memory (one bulk
-// copy) when it fits, otherwise re-read from global memory (L2) on each pass.  Passes over
+// One CTA of PLAN_THREADS threads per row, three per SM.  The row's first
+// PLAN_STAGE_FLOAT4S float4s (all of a Wan-sized row) are staged in shared memory by one
+// bulk copy; the rest of a longer row is re-read from global memory (L2) on each pass.  Passes over
 // the row: staging with the positive count and sum; F at the three fp32 neighbours of
 // lambda0 = s / sum(S) (with the sum of the scores unsaturated at lambda0) -- without
 // saturation lambda* is lambda0 or its upper neighbour, so this one pass brackets it --
