@@ -25,6 +25,7 @@ def _separate(p, Q, K, s, seed, off, S_shape, rows):
 @pytest.mark.parametrize("name,heads,groups,two", [
     ("tiny", None, 2, True), ("tiny", None, 0, True), ("tiny", None, 5, False),
     ("wan13b", [0, 1, 2, 3, 4], 3, True), ("wan13b", [0, 1, 2, 3, 4], 99, True),
+    ("hunyuan13b", [0, 1, 2], 2, True),  # rows longer than the planner's staged prefix
 ])
 def test_select_plan_equals_separate_calls(name, heads, groups, two):
     w = WORKLOADS[name]
