@@ -649,7 +649,21 @@ def run_sweep(args):
     out["all_blocks"] = {"packed_ms": round(t_pk, 3), "dense_path_ms": round(t_dn, 3),
                          "dense_tflops": round(dense_flops / (t_dn * 1e-3) / 1e12, 1),
                          "bitwise_equal": bool(torch.equal(O1, O2))}
-    print(json.dumps(out), flush=True)
+    print(json_line(out), flush=True)
+
+
+def json_line(obj):
+    """The JSON line with every non-finite number as null (a stage-only run leaves the
+    stages it did not time as NaN), so that strict parsers accept it."""
+    def clean(x):
+        if isinstance(x, float) and not math.isfinite(x):
+            return None
+        if isinstance(x, dict):
+            return {k: clean(v) for k, v in x.items()}
+        if isinstance(x, (list, tuple)):
+            return [clean(v) for v in x]
+        return x
+    return json.dumps(clean(obj), allow_nan=False)
 
 
 def run_reference(args, world, rank):
@@ -712,12 +726,12 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         out = run_reference(args, world, rank)
         if out is not None:
-            print(json.dumps(out), flush=True)
+            print(json_line(out), flush=True)
         return
     world, rank, local = dist_setup(args)
     out = run_ours(args, world, rank, local)
     if rank == 0:
-        print(json.dumps(out), flush=True)
+        print(json_line(out), flush=True)
     if world > 1:
         import torch.distributed as dist
 
