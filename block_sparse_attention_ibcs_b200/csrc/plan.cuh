@@ -175,6 +175,13 @@ AB_DEV void block_exscan2_u64(uint64_t v0, uint64_t v1, uint64_t* red0, uint64_t
 // Slots per set: at most PLAN_RED_U uint64 and PLAN_RED_D double values per reduction (kept
 // small: with a staged Wan-sized row, three rows per SM fit in shared memory only so).
 constexpr int PLAN_RED_U = 3, PLAN_RED_D = 1;
+// Three staged rows per SM: each block holds the staged prefix, its static shared memory
+// (the reduction slots, the staging barrier and the Philox word, 16-byte aligned) and the
+// 1 KB the system reserves per block, within the SM's 228 KB.
+static_assert(3 * (PLAN_STAGE_FLOAT4S * 16 +
+                   ((2 * PLAN_RED_U * PLAN_WARPS * 8 + 2 * PLAN_RED_D * PLAN_WARPS * 8 + 8 + 4 + 15) / 16) * 16 +
+                   1024) <= 228 * 1024,
+              "the staged prefix no longer leaves room for three planner rows per SM");
 
 template <int NU, int ND>
 AB_DEV void block_sums(uint64_t (&u)[NU], double (&dv)[ND], uint64_t* ru, double* rd, int& par) {
